@@ -1,0 +1,398 @@
+"""Pins for the CPU oracle: each test ties the oracle to something other than
+itself -- the pages' printed figures, hand-derived examples (tests/golden/),
+library routines that implement the same formats (torch float8_e4m3fn,
+ml_dtypes float4_e2m1fn, torch scaled_dot_product_attention), closed forms,
+invariants and special cases.  CPU only.
+"""
+import math
+
+import ml_dtypes
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import read_golden
+
+E2M1_GRID = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+# --------------------------------------------------------------------------
+# E2M1 element format ("E2M1 + 2レベルスケーリング": sign 1 / exp 2 / mant 1, ~[-6, 6])
+# --------------------------------------------------------------------------
+def test_e2m1_grid_and_range():
+    vals = [oracle.e2m1_value(c) for c in range(16)]
+    assert vals[:8] == E2M1_GRID
+    assert vals[8:] == [-v for v in E2M1_GRID]
+    assert math.copysign(1.0, vals[8]) == -1.0       # code 8 is -0
+    assert max(vals) == 6.0 and min(vals) == -6.0    # the pages' +-6 range
+
+
+def test_e2m1_decode_matches_ml_dtypes():
+    codes = np.arange(16, dtype=np.uint8)
+    lib = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    mine = np.array([oracle.e2m1_value(int(c)) for c in codes])
+    np.testing.assert_array_equal(mine, lib)
+
+
+def _e2m1_sweep():
+    rng = np.random.default_rng(1)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0, 0.5, 1.0], np.float32)
+    near = []
+    for m in mids:
+        bits = m.view(np.uint32).astype(np.int64)
+        near.append((bits + np.arange(-40, 41)).astype(np.uint32).view(np.float32))
+    near = np.concatenate(near)
+    dense = rng.uniform(-8, 8, 200_000).astype(np.float32)
+    tiny = (rng.standard_normal(20_000) * 1e-3).astype(np.float32)
+    big = np.array([7, 100, 1e30, np.inf, 3.4e38], np.float32)
+    every = np.arange(0, 0x41000000, 4099, dtype=np.uint32).view(np.float32)  # [0, 8)
+    allv = np.concatenate([near, -near, dense, tiny, big, -big, every, -every,
+                           np.array([0.0, -0.0], np.float32)])
+    return allv
+
+
+def test_e2m1_encode_matches_ml_dtypes():
+    v = _e2m1_sweep()
+    mine = oracle.e2m1_encode(v)
+    lib = v.astype(ml_dtypes.float4_e2m1fn).view(np.uint8)
+    np.testing.assert_array_equal(mine, lib)
+
+
+def test_e2m1_ties_to_even_and_saturation():
+    v = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.5, 1e9, -0.1, -0.0], np.float32)
+    assert list(oracle.e2m1_encode(v)) == [0, 2, 2, 4, 4, 6, 6, 7, 7, 8, 8]
+
+
+# --------------------------------------------------------------------------
+# E4M3 scale format ("E4M3 FP8" micro-block scale; OCP E4M3FN encoding)
+# --------------------------------------------------------------------------
+def test_e4m3_decode_matches_torch():
+    b = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    lib = b.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = np.array([oracle.e4m3_value(i) for i in range(256)])
+    nan = np.isnan(lib)
+    assert list(np.nonzero(nan)[0]) == [0x7F, 0xFF]
+    np.testing.assert_array_equal(np.isnan(mine), nan)
+    np.testing.assert_array_equal(mine[~nan], lib[~nan])
+    assert mine[0x7E] == 448.0 and mine[0x01] == 2.0 ** -9 and mine[0x08] == 2.0 ** -6
+
+
+def test_e4m3_encode_matches_torch_below_saturation():
+    # every 61st fp32 bit pattern in [0, 464): a dense sweep over all binades,
+    # plus each E4M3 midpoint +-64 ulps (ties), mirrored to negative values.
+    stride = np.arange(0, np.float32(464.0).view(np.uint32), 61, dtype=np.uint32).view(np.float32)
+    grid = torch.arange(0, 127, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn)
+    gv = grid.to(torch.float64).numpy()
+    mids = ((gv[:-1] + gv[1:]) / 2).astype(np.float32)
+    near = np.concatenate([(m.view(np.uint32).astype(np.int64) + np.arange(-64, 65))
+                           .astype(np.uint32).view(np.float32) for m in mids])
+    v = np.concatenate([stride, near, -stride, -near])
+    v = v[np.abs(v) < 464.0]
+    mine = oracle.e4m3_encode(v)
+    lib = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(mine, lib)
+
+
+def test_e4m3_satfinite():
+    v = np.array([448.0, 449.0, 463.99, 464.0, 480.0, 1e6, np.inf, -500.0, -np.inf], np.float32)
+    assert list(oracle.e4m3_encode(v)) == [0x7E] * 7 + [0xFE, 0xFE]
+    assert oracle.e4m3_encode(np.array([np.nan], np.float32))[0] == 0x7F
+
+
+# --------------------------------------------------------------------------
+# Two-level micro-block quantization -- hand-derived examples
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("row", read_golden("quantize_worked.txt"), ids=lambda r: r[0])
+def test_quantize_worked_examples(row):
+    name, st, xs, sb, packed = row
+    x = np.array([float(t) for t in xs.split()], np.float32)
+    assert x.size == 16
+    got_packed, got_sb = oracle.quantize_block(x, np.float32(float(st)))
+    assert got_sb == int(sb, 16)
+    assert [int(b) for b in got_packed] == [int(t, 16) for t in packed.split()]
+
+
+def check_all_quantize_golden():
+    for row in read_golden("quantize_worked.txt"):
+        test_quantize_worked_examples(row)
+
+
+@pytest.mark.parametrize("row", read_golden("dequant_worked.txt"), ids=lambda r: r[0] + r[1])
+def test_dequant_worked_examples(row):
+    code, sb, st, fp8 = row[:4]
+    assert oracle.dequant_fp8(int(code, 16), int(sb, 16), np.float32(float(st))) == int(fp8, 16)
+
+
+# --------------------------------------------------------------------------
+# Quantization invariants (hold for blocks with a normal E4M3 scale)
+# --------------------------------------------------------------------------
+def _random_blocks(n, seed):
+    rng = np.random.default_rng(seed)
+    scale = np.exp(rng.normal(0, 2, (n, 1))).astype(np.float32)
+    return (rng.standard_normal((n, 16)).astype(np.float32) * scale)
+
+
+def _unpack(packed):
+    lo = packed & 0xF
+    hi = packed >> 4
+    return np.stack([lo, hi], -1).reshape(-1)
+
+
+def test_block_invariants():
+    st = np.float32(0.0371)
+    xs = _random_blocks(3000, 7)
+    for x in xs:
+        packed, sb = oracle.quantize_block(x, st)
+        sbv = oracle.e4m3_value(sb)
+        den = np.float32(np.float32(sbv) * st)
+        codes = _unpack(packed)
+        deq = np.array([oracle.e2m1_value(int(c)) for c in codes]) * float(den)
+        if sbv < 2.0 ** -6:      # subnormal or zero scale: compared to the oracle only
+            continue
+        if np.abs(x).max() / (6.0 * float(st)) > 448.0:   # beyond the calibrated range
+            assert sb == 0x7E                             # the scale saturates ...
+            continue                                      # ... and the bound does not apply
+        # the block's largest element takes the largest code +-6 ...
+        imax = int(np.argmax(np.abs(x)))
+        assert abs(oracle.e2m1_value(int(codes[imax]))) == 6.0
+        # ... every element is reconstructed within one scale step ...
+        err = np.abs(x.astype(np.float64) - deq)
+        assert np.all(err <= 1.0 * float(den) * (1 + 1e-6))
+        # ... and within a quarter step below the 1.75 threshold
+        small = np.abs(x / den) < 1.75
+        assert np.all(err[small] <= 0.25 * float(den) * (1 + 1e-6))
+        # sign symmetry: negating x flips code signs only
+        packed_n, sb_n = oracle.quantize_block(-x, st)
+        assert sb_n == sb
+        np.testing.assert_array_equal(_unpack(packed_n), codes ^ 0x8)
+
+
+def test_grid_data_round_trip():
+    rng = np.random.default_rng(3)
+    st = np.float32(0.5)
+    for _ in range(500):
+        sb = int(rng.integers(0x10, 0x70))         # normal scales
+        codes = rng.integers(0, 16, 16).astype(np.uint8)
+        codes[int(rng.integers(16))] = 0x7 | (0x8 if rng.random() < 0.5 else 0)
+        den = np.float32(np.float32(oracle.e4m3_value(sb)) * st)
+        x = np.array([oracle.e2m1_value(int(c)) for c in codes], np.float32) * den
+        packed, sb2 = oracle.quantize_block(x, st)
+        assert sb2 == sb
+        got = _unpack(packed)
+        # zero codes may come back as +0 or -0 depending on the sign of 0*den
+        np.testing.assert_array_equal(got & 0x7, codes & 0x7)
+        nz = (codes & 0x7) != 0
+        np.testing.assert_array_equal(got[nz], codes[nz])
+
+
+# --------------------------------------------------------------------------
+# Calibration (level-2 FP32 tensor scale)
+# --------------------------------------------------------------------------
+def test_tensor_scale():
+    st, s = oracle.tensor_scale(np.array([1.0, -2688.0, 3.0], np.float32))
+    assert st == 0 and s == np.float32(1.0)
+    st, s = oracle.tensor_scale(np.array([0.5, -0.25], np.float32))
+    assert s == np.float32(0.5) / np.float32(2688.0)
+    assert oracle.tensor_scale(np.zeros(5, np.float32)) == (0, np.float32(1.0))
+    assert oracle.tensor_scale(np.array([1, np.nan], np.float32))[0] == 4
+    assert oracle.tensor_scale(np.array([1, -np.inf], np.float32))[0] == 4
+    # with s_tensor from amax the largest block scale is exactly 448 (no saturation)
+    x = np.zeros(16, np.float32)
+    x[3] = -123.25
+    _, s = oracle.tensor_scale(x)
+    packed, sb = oracle.quantize_block(x, s)
+    assert sb == 0x7E and (_unpack(packed)[3]) == 0xF
+
+
+# --------------------------------------------------------------------------
+# Append into the cache planes
+# --------------------------------------------------------------------------
+def test_quantize_append_placement_and_capacity():
+    rng = np.random.default_rng(5)
+    B, n_new, H, D, S = 3, 4, 2, 32, 16
+    x = rng.standard_normal((B, n_new, H, D)).astype(np.float32)
+    codes, scales = oracle.new_planes(B, H, S, D)
+    start = np.array([0, 5, 12], np.int32)
+    assert oracle.quantize_append(x, start, 0.01, codes, scales) == 0
+    for b in range(B):
+        for t in range(n_new):
+            for h in range(H):
+                for blk in range(D // 16):
+                    p, sb = oracle.quantize_block(x[b, t, h, 16 * blk:16 * blk + 16], 0.01)
+                    slot = start[b] + t
+                    assert scales[b, h, slot, blk] == sb
+                    np.testing.assert_array_equal(codes[b, h, slot, 8 * blk:8 * blk + 8], p)
+    untouched = np.ones(S, bool)
+    untouched[5:9] = False
+    assert not codes[1, :, untouched].any() and not scales[1, :, untouched].any()
+    # overflow of one sequence is reported and leaves that sequence untouched
+    codes2, scales2 = oracle.new_planes(B, H, S, D)
+    assert oracle.quantize_append(x, np.array([0, 13, 1], np.int32), 0.01, codes2, scales2) == 3
+    assert not codes2[1].any() and codes2[0].any() and codes2[2].any()
+
+
+def test_dequant_planes_matches_elementwise():
+    rng = np.random.default_rng(9)
+    B, H, D, S = 2, 1, 32, 8
+    codes = rng.integers(0, 256, (B, H, S, D // 2)).astype(np.uint8)
+    scales = rng.integers(0, 0x7F, (B, H, S, D // 16)).astype(np.uint8)
+    lens = np.array([8, 3], np.int32)
+    out = oracle.dequant_planes(codes, scales, 0.013, lens)
+    for b in range(B):
+        for t in range(S):
+            for d in range(D):
+                byte = codes[b, 0, t, d // 2]
+                c = byte & 0xF if d % 2 == 0 else byte >> 4
+                want = oracle.dequant_fp8(int(c), int(scales[b, 0, t, d // 16]), 0.013) \
+                    if t < lens[b] else 0
+                assert out[b, 0, t, d] == want
+
+
+def test_dequant_fp8_sign_and_value():
+    rng = np.random.default_rng(11)
+    for _ in range(2000):
+        c = int(rng.integers(0, 16))
+        sb = int(rng.integers(0, 0x7F))
+        st = np.float32(np.exp(rng.normal(-4, 2)))
+        e = oracle.dequant_fp8(c, sb, st)
+        assert (e >> 7) == (c >> 3)                       # sign copied
+        exact = abs(oracle.e2m1_value(c)) * oracle.e4m3_value(sb) * float(st)
+        got = abs(oracle.e4m3_value(e))
+        if 2.0 ** -6 <= exact <= 448:                     # normal E4M3 range: 2^-4 relative
+            assert abs(got - exact) <= exact * 2.0 ** -4 * (1 + 1e-6)
+        elif exact < 2.0 ** -6:                           # subnormal: half a step absolute
+            assert abs(got - exact) <= 2.0 ** -10 * (1 + 1e-6)
+        else:
+            assert got == 448.0
+
+
+# --------------------------------------------------------------------------
+# Attention (fp64) -- library routine, closed forms and special cases
+# --------------------------------------------------------------------------
+def _rand_fp8_planes(rng, B, H_kv, S, D):
+    return (rng.integers(0, 256, (B, H_kv, S, D)).astype(np.uint8),
+            rng.integers(0, 256, (B, H_kv, S, D)).astype(np.uint8))
+
+
+def _fp8_values(p):
+    v = torch.from_numpy(p).view(torch.float8_e4m3fn).to(torch.float64)
+    return torch.nan_to_num(v, nan=0.0)
+
+
+def _sanitize(p):
+    p = p.copy()
+    p[(p & 0x7F) == 0x7F] = 0x00          # no NaN encodings in the cache
+    return p
+
+
+def test_attention_matches_torch_sdpa_gqa():
+    rng = np.random.default_rng(13)
+    B, H_q, H_kv, S, D = 3, 6, 2, 40, 32
+    k8, v8 = _rand_fp8_planes(rng, B, H_kv, S, D)
+    k8, v8 = _sanitize(k8) & 0xBF, _sanitize(v8)      # keep K moderate
+    q = rng.standard_normal((B, H_q, D)).astype(np.float32)
+    lens = np.array([40, 1, 17], np.int32)
+    got = oracle.decode_attention_fp8(q, k8, v8, lens)
+    K, V = _fp8_values(k8), _fp8_values(v8)
+    g = H_q // H_kv
+    for b in range(B):
+        L = int(lens[b])
+        qt = torch.from_numpy(q[b]).to(torch.float64).view(H_q, 1, D)
+        Kt = K[b, :, :L].repeat_interleave(g, 0)
+        Vt = V[b, :, :L].repeat_interleave(g, 0)
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt).view(H_q, D)
+        np.testing.assert_allclose(got[b], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(17)
+    B, H_q, H_kv, S, D = 1, 2, 1, 24, 16
+    k8, v8 = _rand_fp8_planes(rng, B, H_kv, S, D)
+    k8, v8 = _sanitize(k8), _sanitize(v8)
+    V = _fp8_values(v8).numpy()
+    # q = 0: uniform weights, output = mean of the cached V rows
+    q0 = np.zeros((B, H_q, D), np.float32)
+    out = oracle.decode_attention_fp8(q0, k8, v8, np.array([S], np.int32))
+    np.testing.assert_allclose(out[0, 0], V[0, 0].mean(0), rtol=1e-12, atol=1e-12)
+    # one cached token: output = that V row
+    q = rng.standard_normal((B, H_q, D)).astype(np.float32)
+    out = oracle.decode_attention_fp8(q, k8, v8, np.array([1], np.int32))
+    np.testing.assert_array_equal(out[0, 1], V[0, 0, 0])
+    # empty sequence: zero row
+    out = oracle.decode_attention_fp8(q, k8, v8, np.array([0], np.int32))
+    assert not out.any()
+    # two tokens: logistic weights sigma(s0 - s1)
+    k2 = np.zeros((1, 1, 2, D), np.uint8)
+    k2[0, 0, 0, 0] = 0x38                     # k0 = e0 (1.0)
+    v2 = np.zeros((1, 1, 2, D), np.uint8)
+    v2[0, 0, 0, 0] = 0x40                     # v0 = 2 e0
+    v2[0, 0, 1, 1] = 0x38                     # v1 = e1
+    qq = np.zeros((1, 1, D), np.float32)
+    qq[0, 0, 0] = 3.0
+    out = oracle.decode_attention_fp8(qq, k2, v2, np.array([2], np.int32))
+    s0 = 3.0 / math.sqrt(D)
+    w0 = 1.0 / (1.0 + math.exp(-s0))
+    np.testing.assert_allclose(out[0, 0, :2], [2 * w0, 1 - w0], rtol=1e-14)
+    # explicit softmax_scale replaces 1/sqrt(D)
+    out = oracle.decode_attention_fp8(qq, k2, v2, np.array([2], np.int32), softmax_scale=0.5)
+    w0 = 1.0 / (1.0 + math.exp(-1.5))
+    np.testing.assert_allclose(out[0, 0, :2], [2 * w0, 1 - w0], rtol=1e-14)
+
+
+def test_attention_token_permutation_invariance():
+    rng = np.random.default_rng(19)
+    B, H_q, H_kv, S, D = 1, 4, 2, 30, 16
+    k8, v8 = _rand_fp8_planes(rng, B, H_kv, S, D)
+    k8, v8 = _sanitize(k8) & 0xBF, _sanitize(v8)
+    q = rng.standard_normal((B, H_q, D)).astype(np.float32)
+    perm = rng.permutation(S)
+    a = oracle.decode_attention_fp8(q, k8, v8, np.array([S], np.int32))
+    b = oracle.decode_attention_fp8(q, k8[:, :, perm], v8[:, :, perm], np.array([S], np.int32))
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_nvfp4_composes_dequant_and_fp8_attention():
+    rng = np.random.default_rng(23)
+    B, H_q, H_kv, S, D = 2, 4, 2, 20, 32
+    x_k = rng.standard_normal((B, S, H_kv, D)).astype(np.float32)
+    x_v = rng.standard_normal((B, S, H_kv, D)).astype(np.float32)
+    _, sk = oracle.tensor_scale(x_k)
+    _, sv = oracle.tensor_scale(x_v)
+    kc, ks = oracle.new_planes(B, H_kv, S, D)
+    vc, vs = oracle.new_planes(B, H_kv, S, D)
+    zero = np.zeros(B, np.int32)
+    assert oracle.quantize_append(x_k, zero, sk, kc, ks) == 0
+    assert oracle.quantize_append(x_v, zero, sv, vc, vs) == 0
+    lens = np.array([20, 7], np.int32)
+    q = rng.standard_normal((B, H_q, D)).astype(np.float32)
+    full = oracle.decode_attention_nvfp4(q, kc, ks, vc, vs, sk, sv, lens)
+    k8 = oracle.dequant_planes(kc, ks, sk, lens)
+    v8 = oracle.dequant_planes(vc, vs, sv, lens)
+    two = oracle.decode_attention_fp8(q, k8, v8, lens)
+    np.testing.assert_array_equal(full, two)
+    # and NVFP4 attention stays close to attention on the unquantized inputs
+    Kx = torch.from_numpy(x_k).permute(0, 2, 1, 3).to(torch.float64)
+    Vx = torch.from_numpy(x_v).permute(0, 2, 1, 3).to(torch.float64)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q).to(torch.float64)[:, :, None, :],
+        Kx.repeat_interleave(2, 1)[:, :, :20], Vx.repeat_interleave(2, 1)[:, :, :20])[0, :, 0]
+    assert np.abs(full[0] - ref.numpy()).max() < 0.3
+
+
+# --------------------------------------------------------------------------
+# Memory model ("KV Cacheのメモリボトルネック" formula, "メモリ削減効果" table)
+# --------------------------------------------------------------------------
+def test_memory_ratios_match_pages():
+    printed = {r[0]: (float(r[1]), float(r[2])) for r in read_golden("memory_ratios.txt")}
+    bits = oracle.nvfp4_bits_per_element()
+    assert bits == 4.5
+    args = (80, 8, 128, 65536, 4)          # layers, n_h, d_h, s, b
+    fp16 = oracle.kv_bytes(*args, 16)
+    fp8 = oracle.kv_bytes(*args, 8)
+    nv = oracle.kv_bytes(*args, bits)
+    assert fp16 == 2 * 80 * 8 * 128 * 65536 * 4 * 2
+    for name, val in [("ratio_vs_fp16", fp16 / nv), ("ratio_vs_fp8", fp8 / nv),
+                      ("reduction_vs_fp16", 1 - nv / fp16), ("fraction_of_fp8", nv / fp8)]:
+        want, tol = printed[name]
+        assert abs(val - want) <= tol, (name, val, want)
