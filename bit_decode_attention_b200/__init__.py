@@ -1,0 +1,160 @@
+"""bit_decode_attention_b200 -- NVFP4 KV cache with fused NVFP4 -> FP8 decode
+attention for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI of libnvfp4kv.so (include/nvfp4kv.h).
+The functions below carry the C names and only marshal arguments: torch
+tensors supply device memory and the current CUDA stream, every step of the
+computation runs in the library's kernels.  There is no CPU path.
+
+Formats and flow follow "NVIDIA解説: NVFP4 KV Cacheで長コンテキストLLM推論を最適化"
+(sections "E2M1 + 2レベルスケーリング" and "量子化・逆量子化フロー").
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+from typing import Optional
+
+import torch
+
+from . import _native
+from ._native import (NVFP4_ERR_CAPACITY, NVFP4_ERR_INVALID_ARG, NVFP4_ERR_NONFINITE,  # noqa: F401
+                      NVFP4_ERR_TIMEOUT, NVFP4_ERR_UNSUPPORTED, NVFP4_ERR_WORKSPACE, NVFP4_OK,
+                      NativeError)
+
+__all__ = [
+    "KVPlane", "nvfp4_cache_bytes", "nvfp4_calib_tensor_scale", "nvfp4_kv_quantize_append",
+    "nvfp4_kv_dequant_fp8", "nvfp4_decode_attention_workspace", "nvfp4_decode_attention",
+    "nvfp4_version", "NativeError",
+]
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return _native.NVFP4_IN_BF16
+    if t.dtype == torch.float32:
+        return _native.NVFP4_IN_F32
+    raise TypeError("inputs must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+@dataclasses.dataclass
+class KVPlane:
+    """One NVFP4 cache plane (K or V) in device memory.
+
+    codes  uint8 [B][H_kv][S_max][D/2]  (element 2j low nibble of byte j)
+    scales uint8 [B][H_kv][S_max][D/16] (one E4M3 byte per 16 elements)
+    """
+    codes: torch.Tensor
+    scales: torch.Tensor
+
+    @classmethod
+    def allocate(cls, B: int, H_kv: int, S_max: int, D: int, device="cuda") -> "KVPlane":
+        codes = torch.zeros(B, H_kv, S_max, D // 2, dtype=torch.uint8, device=device)
+        scales = torch.zeros(B, H_kv, S_max, D // 16, dtype=torch.uint8, device=device)
+        return cls(codes, scales)
+
+    @property
+    def shape(self):
+        B, H, S, Dh = self.codes.shape
+        return B, H, S, 2 * Dh
+
+    def struct(self) -> _native.KVPlaneStruct:
+        B, H, S, D = self.shape
+        return _native.KVPlaneStruct(self.codes.data_ptr(), self.scales.data_ptr(), B, H, S, D)
+
+
+def nvfp4_version() -> str:
+    return _native.lib().nvfp4_version().decode()
+
+
+def nvfp4_cache_bytes(B: int, H_kv: int, S_max: int, D: int) -> int:
+    return int(_native.lib().nvfp4_cache_bytes(B, H_kv, S_max, D))
+
+
+def nvfp4_calib_tensor_scale(x: torch.Tensor, s_tensor: Optional[torch.Tensor] = None,
+                             status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Per-tensor scale fl32(amax / 2688) as a 1-element device float tensor."""
+    _need_cuda(x)
+    if s_tensor is None:
+        s_tensor = torch.empty(1, dtype=torch.float32, device=x.device)
+    st = _native.lib().nvfp4_calib_tensor_scale(_ptr(x), _dtype_code(x), x.numel(), _ptr(s_tensor),
+                                                _ptr(status), _stream(stream))
+    _native.check("nvfp4_calib_tensor_scale", st)
+    return s_tensor
+
+
+def nvfp4_kv_quantize_append(x_new: torch.Tensor, start_pos: torch.Tensor, s_tensor: torch.Tensor,
+                             plane: KVPlane, new_lens: Optional[torch.Tensor] = None,
+                             status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Quantize x_new [B][n_new][H_kv][D] and write it at slots start_pos[b]... of `plane`."""
+    _need_cuda(x_new, start_pos, s_tensor, new_lens, status)
+    n_new = x_new.shape[1]
+    pl = plane.struct()
+    st = _native.lib().nvfp4_kv_quantize_append(_ptr(x_new), _dtype_code(x_new), n_new,
+                                                _ptr(start_pos), _ptr(new_lens), _ptr(s_tensor),
+                                                ctypes.byref(pl), _ptr(status), _stream(stream))
+    _native.check("nvfp4_kv_quantize_append", st)
+
+
+def nvfp4_kv_dequant_fp8(plane: KVPlane, s_tensor: torch.Tensor, seq_lens: torch.Tensor,
+                         out: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """E4M3 bytes [B][H_kv][S_max][D] for the first seq_lens[b] slots."""
+    _need_cuda(s_tensor, seq_lens, out, status)
+    B, H, S, D = plane.shape
+    if out is None:
+        out = torch.zeros(B, H, S, D, dtype=torch.uint8, device=plane.codes.device)
+    pl = plane.struct()
+    st = _native.lib().nvfp4_kv_dequant_fp8(ctypes.byref(pl), _ptr(s_tensor), _ptr(seq_lens),
+                                            _ptr(out), _ptr(status), _stream(stream))
+    _native.check("nvfp4_kv_dequant_fp8", st)
+    return out
+
+
+def nvfp4_decode_attention_workspace(B: int, H_q: int, H_kv: int, D: int) -> int:
+    return int(_native.lib().nvfp4_decode_attention_workspace(B, H_q, H_kv, D))
+
+
+def new_workspace(B: int, H_q: int, H_kv: int, D: int, device="cuda") -> torch.Tensor:
+    """Zero-filled workspace for nvfp4_decode_attention (reusable across calls)."""
+    n = nvfp4_decode_attention_workspace(B, H_q, H_kv, D)
+    if n == 0:
+        raise ValueError("unsupported attention shape")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def nvfp4_decode_attention(q: torch.Tensor, k: KVPlane, v: KVPlane, s_tensor_k: torch.Tensor,
+                           s_tensor_v: torch.Tensor, seq_lens: torch.Tensor,
+                           softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                           workspace: Optional[torch.Tensor] = None,
+                           status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """softmax(q K^T * scale) V over the NVFP4 cache; q [B][H_q][D] -> fp32 [B][H_q][D]."""
+    _need_cuda(q, s_tensor_k, s_tensor_v, seq_lens, out, workspace, status)
+    B, H_q, D = q.shape
+    Bk, H_kv, S, Dk = k.shape
+    if out is None:
+        out = torch.empty(B, H_q, D, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(B, H_q, H_kv, D, device=q.device)
+    kp, vp = k.struct(), v.struct()
+    st = _native.lib().nvfp4_decode_attention(
+        _ptr(q), _dtype_code(q), H_q, ctypes.byref(kp), ctypes.byref(vp), _ptr(s_tensor_k),
+        _ptr(s_tensor_v), _ptr(seq_lens), ctypes.c_float(softmax_scale), _ptr(out),
+        _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
+    _native.check("nvfp4_decode_attention", st)
+    return out

@@ -1,0 +1,180 @@
+// nvfp4kv_api.cu -- the extern "C" entry points of libnvfp4kv.so declared in
+// include/nvfp4kv.h: argument validation, workspace layout and launches.
+// Every call is asynchronous on the caller's stream and allocates nothing.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "../../include/nvfp4kv.h"
+#include "nvfp4kv_internal.h"
+
+namespace nvfp4kv {
+
+int device_sm_count() {
+    static int cached_dev = -1;
+    static int cached_count = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev != cached_dev) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached_count = n;
+        cached_dev = dev;
+    }
+    return cached_count;
+}
+
+AttnWorkspace attention_workspace(int B, int Hq, int Hkv, int D) {
+    AttnWorkspace w{};
+    const int g = Hq / Hkv;
+    w.grid = kCtasPerSm * device_sm_count();
+    w.counters_bytes = ((size_t)B * Hkv * sizeof(int32_t) + 255) / 256 * 256;
+    w.partial_floats = (size_t)2 * w.grid * g * (D + 2);
+    w.total_bytes = w.counters_bytes + w.partial_floats * sizeof(float);
+    return w;
+}
+
+}  // namespace nvfp4kv
+
+namespace {
+
+using namespace nvfp4kv;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool plane_ok(const nvfp4_kv_plane* pl) {
+    if (pl == nullptr || pl->codes == nullptr || pl->scales == nullptr) return false;
+    if (pl->B < 0 || pl->H_kv <= 0 || pl->S_max <= 0 || (pl->S_max % 16) != 0) return false;
+    if (pl->D != 64 && pl->D != 128) return false;
+    if (!aligned16(pl->codes) || !aligned16(pl->scales)) return false;
+    return true;
+}
+
+nvfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* nvfp4_status_string(int status) {
+    switch (status) {
+        case NVFP4_OK: return "ok";
+        case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+        case NVFP4_ERR_UNSUPPORTED: return "unsupported";
+        case NVFP4_ERR_CAPACITY: return "sequence past cache capacity";
+        case NVFP4_ERR_NONFINITE: return "non-finite value or scale";
+        case NVFP4_ERR_CUDA: return "CUDA error";
+        case NVFP4_ERR_TIMEOUT: return "device wait timed out";
+        case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+const char* nvfp4_version(void) { return "nvfp4kv 0.1.0 (sm_100a)"; }
+
+size_t nvfp4_cache_bytes(int B, int H_kv, int S_max, int D) {
+    if (B < 0 || H_kv <= 0 || S_max < 0 || D <= 0 || (D % 16) != 0) return 0;
+    return (size_t)B * H_kv * S_max * (size_t)(D / 2 + D / 16);
+}
+
+nvfp4_status nvfp4_calib_tensor_scale(const void* x, nvfp4_dtype dtype, int64_t n,
+                                      float* d_s_tensor, int32_t* d_status, nvfp4_stream_t stream) {
+    if (d_s_tensor == nullptr || n < 0 || (n > 0 && x == nullptr)) return NVFP4_ERR_INVALID_ARG;
+    if (dtype != NVFP4_IN_BF16 && dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
+    const size_t esz = dtype == NVFP4_IN_F32 ? 4 : 2;
+    if ((reinterpret_cast<uintptr_t>(x) % esz) != 0) return NVFP4_ERR_INVALID_ARG;
+    return from_cuda(launch_calib(x, dtype == NVFP4_IN_F32, n, d_s_tensor, d_status,
+                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_kv_quantize_append(const void* x_new, nvfp4_dtype dtype, int n_new,
+                                      const int32_t* d_start_pos, int32_t* d_new_lens,
+                                      const float* d_s_tensor, const nvfp4_kv_plane* plane,
+                                      int32_t* d_status, nvfp4_stream_t stream) {
+    if (!plane_ok(plane) || n_new < 0 || d_s_tensor == nullptr || d_start_pos == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (dtype != NVFP4_IN_BF16 && dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
+    if (d_new_lens != nullptr && d_new_lens == d_start_pos) return NVFP4_ERR_INVALID_ARG;
+    if (n_new == 0 || plane->B == 0) return NVFP4_OK;
+    if (x_new == nullptr || !aligned16(x_new)) return NVFP4_ERR_INVALID_ARG;
+    return from_cuda(launch_quantize_append(x_new, dtype == NVFP4_IN_F32, n_new, d_start_pos,
+                                            d_new_lens, d_s_tensor, *plane, d_status,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_kv_dequant_fp8(const nvfp4_kv_plane* plane, const float* d_s_tensor,
+                                  const int32_t* d_seq_lens, uint8_t* out_e4m3, int32_t* d_status,
+                                  nvfp4_stream_t stream) {
+    if (!plane_ok(plane) || d_s_tensor == nullptr || d_seq_lens == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (plane->B == 0) return NVFP4_OK;
+    if (out_e4m3 == nullptr || !aligned16(out_e4m3)) return NVFP4_ERR_INVALID_ARG;
+    return from_cuda(launch_dequant_fp8(*plane, d_s_tensor, d_seq_lens, out_e4m3, d_status,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t nvfp4_decode_attention_workspace(int B, int H_q, int H_kv, int D) {
+    if (B < 0 || H_kv <= 0 || H_q <= 0 || (H_q % H_kv) != 0 || H_q / H_kv > 16) return 0;
+    if (D != 64 && D != 128) return 0;
+    return attention_workspace(B, H_q, H_kv, D).total_bytes;
+}
+
+nvfp4_status nvfp4_decode_attention(const void* q, nvfp4_dtype q_dtype, int H_q,
+                                    const nvfp4_kv_plane* k, const nvfp4_kv_plane* v,
+                                    const float* d_s_tensor_k, const float* d_s_tensor_v,
+                                    const int32_t* d_seq_lens, float softmax_scale, float* out,
+                                    void* workspace, size_t workspace_bytes, int32_t* d_status,
+                                    nvfp4_stream_t stream) {
+    if (!plane_ok(k) || !plane_ok(v)) return NVFP4_ERR_INVALID_ARG;
+    if (k->B != v->B || k->H_kv != v->H_kv || k->S_max != v->S_max || k->D != v->D)
+        return NVFP4_ERR_INVALID_ARG;
+    if (q_dtype != NVFP4_IN_BF16 && q_dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
+    if (H_q <= 0 || (H_q % k->H_kv) != 0) return NVFP4_ERR_INVALID_ARG;
+    if (H_q / k->H_kv > 16) return NVFP4_ERR_UNSUPPORTED;
+    if (d_s_tensor_k == nullptr || d_s_tensor_v == nullptr || d_seq_lens == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!(std::isfinite(softmax_scale)) || softmax_scale < 0.0f) return NVFP4_ERR_INVALID_ARG;
+    const int B = k->B;
+    if (B == 0) return NVFP4_OK;
+    if (q == nullptr || out == nullptr || !aligned16(q)) return NVFP4_ERR_INVALID_ARG;
+    const AttnWorkspace ws = attention_workspace(B, H_q, k->H_kv, k->D);
+    if (workspace == nullptr || workspace_bytes < ws.total_bytes || !aligned16(workspace))
+        return NVFP4_ERR_WORKSPACE;
+
+    const int D = k->D;
+    const size_t esz = q_dtype == NVFP4_IN_F32 ? 4 : 2;
+    const size_t plane_tok = (size_t)k->H_kv * k->S_max;  // token slots per sequence
+    AttnLaunch a{};
+    a.q_f32 = q_dtype == NVFP4_IN_F32;
+    a.Hq = H_q;
+    a.Hkv = k->H_kv;
+    a.S_max = k->S_max;
+    a.D = D;
+    a.st_k = d_s_tensor_k;
+    a.st_v = d_s_tensor_v;
+    a.softmax_scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt((float)D);
+    a.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ws.counters_bytes);
+    a.status = d_status;
+    a.grid = ws.grid;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    for (int b0 = 0; b0 < B; b0 += kMaxBatchPerLaunch) {
+        const int nb = (B - b0) < kMaxBatchPerLaunch ? (B - b0) : kMaxBatchPerLaunch;
+        a.B = nb;
+        a.q = static_cast<const uint8_t*>(q) + (size_t)b0 * H_q * D * esz;
+        a.kc = k->codes + (size_t)b0 * plane_tok * (D / 2);
+        a.ks = k->scales + (size_t)b0 * plane_tok * (D / 16);
+        a.vc = v->codes + (size_t)b0 * plane_tok * (D / 2);
+        a.vs = v->scales + (size_t)b0 * plane_tok * (D / 16);
+        a.seq_lens = d_seq_lens + b0;
+        a.out = out + (size_t)b0 * H_q * D;
+        a.counters = static_cast<int32_t*>(workspace) + (size_t)b0 * k->H_kv;
+        cudaError_t e = launch_decode_attention(a, s);
+        if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_OK;
+}
+
+}  // extern "C"

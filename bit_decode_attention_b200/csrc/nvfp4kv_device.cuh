@@ -1,0 +1,227 @@
+// nvfp4kv_device.cuh -- device-side building blocks of libnvfp4kv.so:
+// E4M3 / E2M1 conversions written from the format definitions, the per-block
+// FP8 lookup used to dequantize NVFP4 codes, and thin PTX wrappers for the
+// sm_100a instructions the kernels use (mbarrier, bulk async copy, warp MMA,
+// movmatrix).
+//
+// Formats ("NVIDIA解説: NVFP4 KV Cacheで長コンテキストLLM推論を最適化",
+// section "E2M1 + 2レベルスケーリング"): E2M1 elements (sign/exp2/mant1,
+// range +-6), one E4M3 scale per 16 elements, one fp32 tensor scale.
+// E4M3 is the OCP E4M3FN byte: bias 7, largest finite 448, S.1111.111 = NaN.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/nvfp4kv.h"
+
+namespace nvfp4kv {
+
+// ---------------------------------------------------------------------------
+// status word: the first error wins
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void report(int32_t* status, int32_t code) {
+    if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+// ---------------------------------------------------------------------------
+// E4M3 (E4M3FN) conversions
+// ---------------------------------------------------------------------------
+// float -> E4M3 byte, round to nearest (ties to even), finite overflow
+// saturates to +-448, NaN -> 0x7F.  Integer rounding of the fp32 bit pattern:
+// for normal results the 23-bit fraction is rounded to 3 bits (carry into the
+// exponent is the correct next binade); below 2^-6 the result is a multiple
+// of 2^-9 and |v| * 2^9 is rounded to an integer 0..8 (8 encodes 2^-6).
+__device__ __forceinline__ uint32_t e4m3_from_float(float v) {
+    const uint32_t bits = __float_as_uint(v);
+    const uint32_t sign = (bits >> 24) & 0x80u;
+    const uint32_t a = bits & 0x7FFFFFFFu;
+    if (a > 0x7F800000u) return 0x7Fu;                 // NaN
+    if (a >= 0x43E00000u) return sign | 0x7Eu;         // |v| >= 448 (incl. inf)
+    if (a >= 0x3C800000u) {                            // |v| >= 2^-6: normal
+        const uint32_t odd = (a >> 20) & 1u;
+        uint32_t r = (a + 0x7FFFFu + odd) >> 20;       // exp32:3 | mant3, rounded
+        r -= (127u - 7u) << 3;                         // rebias 127 -> 7
+        return sign | (r > 0x7Eu ? 0x7Eu : r);
+    }
+    const float scaled = __uint_as_float(a) * 512.0f;  // exact (power of two)
+    return sign | __float2uint_rn(scaled);             // 0..8, ties to even
+}
+
+// E4M3 byte (not NaN) -> float, exact.
+__device__ __forceinline__ float e4m3_to_float(uint32_t b) {
+    const uint32_t e = (b >> 3) & 0xFu;
+    const uint32_t m = b & 7u;
+    const float mag = (e == 0) ? (float)m * 0.001953125f                       // m * 2^-9
+                               : __uint_as_float(((e + 120u) << 23) | (m << 20));
+    return (b & 0x80u) ? -mag : mag;
+}
+
+// ---------------------------------------------------------------------------
+// E2M1 conversions
+// ---------------------------------------------------------------------------
+// |code| -> value: 0, 0.5, 1, 1.5, 2, 3, 4, 6
+__device__ __forceinline__ float e2m1_magnitude(uint32_t m3) {
+    // exponent field e = m3 >> 1, mantissa bit = m3 & 1 (bias 1; e == 0 subnormal)
+    const uint32_t e = m3 >> 1, mb = m3 & 1u;
+    return e == 0 ? 0.5f * (float)mb : (1.0f + 0.5f * (float)mb) * (float)(1u << (e - 1));
+}
+
+// float -> E2M1 code: nearest grid value, ties to the even code, saturating at
+// +-6; the sign bit is copied (negative values rounding to 0 give 0x8).  The
+// comparisons are against the exact midpoints of the grid, strict where the
+// lower neighbour has the even code and inclusive where the upper one has.
+__device__ __forceinline__ uint32_t e2m1_from_float(float y) {
+    const float a = fabsf(y);
+    uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) +
+                 (a > 2.5f) + (a >= 3.5f) + (a > 5.0f);
+    return c | ((__float_as_uint(y) >> 28) & 0x8u);
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4 -> FP8 lookup
+// ---------------------------------------------------------------------------
+// The FP8 value of a code depends only on its 3-bit magnitude, the block's
+// scale byte and the tensor scale.  lut_entry(sb, m, st) is that value for one
+// magnitude; a block's 8 entries fit two 32-bit words, which `byte_perm` then
+// indexes with four 3-bit selectors at a time.
+__device__ __forceinline__ uint32_t lut_entry(uint32_t sb, uint32_t m3, float s_tensor) {
+    if ((sb & 0x7Fu) == 0x7Fu) return 0u;                    // never written by quantize
+    const float prod = __fmul_rn(e2m1_magnitude(m3), e4m3_to_float(sb & 0x7Fu)); // exact
+    return e4m3_from_float(__fmul_rn(prod, s_tensor));
+}
+
+// Dequantize 8 packed codes (one 32-bit word; element k in nibble k) to 8 FP8
+// bytes with the block's lookup words (lut_lo = magnitudes 0..3, lut_hi =
+// 4..7).  out_lo = elements 0..3, out_hi = elements 4..7 (byte k = element k).
+//   - magnitudes: byte_perm selects one lookup byte per 3-bit selector;
+//   - signs: nibble msb k sits at bit 4k+3 and must land at bit 8k+7; the
+//     byte permutes of (x << 4, x) move bits 3/7/11/15 (19/23/27/31) there.
+__device__ __forceinline__ void dequant_word(uint32_t x, uint32_t lut_lo, uint32_t lut_hi,
+                                             uint32_t& out_lo, uint32_t& out_hi) {
+    const uint32_t sel_lo = x & 0x7777u;
+    const uint32_t sel_hi = (x >> 16) & 0x7777u;
+    const uint32_t mag_lo = __byte_perm(lut_lo, lut_hi, sel_lo);
+    const uint32_t mag_hi = __byte_perm(lut_lo, lut_hi, sel_hi);
+    const uint32_t xs = x << 4;
+    const uint32_t sgn_lo = __byte_perm(xs, x, 0x5140u);
+    const uint32_t sgn_hi = __byte_perm(xs, x, 0x7362u);
+    out_lo = mag_lo | (sgn_lo & 0x80808080u);
+    out_hi = mag_hi | (sgn_hi & 0x80808080u);
+}
+
+// ---------------------------------------------------------------------------
+// small PTX wrappers (sm_90+ / sm_100a)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete; give up after
+// `limit` polls (each poll may suspend the thread for a short while).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t limit) {
+    for (uint32_t i = 0; i < limit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+// dst, src and bytes must be multiples of 16.  No cluster multicast.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Order this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy (bulk copy) writes to the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Two E4M3 bytes (lo, hi of a 16-bit value) -> f16x2 (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t lo16_to_f16x2(uint32_t x) {
+    return e4m3x2_to_f16x2(static_cast<uint16_t>(x & 0xFFFFu));
+}
+__device__ __forceinline__ uint32_t hi16_to_f16x2(uint32_t x) {
+    return e4m3x2_to_f16x2(static_cast<uint16_t>(x >> 16));
+}
+
+// Two floats -> f16x2 (lo in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ float f16_lo_to_float(uint32_t x) {
+    float f;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.f32.f16 %0, l;\n\t}" : "=f"(f) : "r"(x));
+    return f;
+}
+__device__ __forceinline__ float f16_hi_to_float(uint32_t x) {
+    float f;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.f32.f16 %0, h;\n\t}" : "=f"(f) : "r"(x));
+    return f;
+}
+
+// 8x8 b16 matrix transpose across the warp (fragment layout: lane holds row
+// lane/4, columns 2*(lane%4), +1).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t r;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+    return r;
+}
+
+// D += A(16x16, f16, row) * B(16x8, f16, col), fp32 accumulate.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+}  // namespace nvfp4kv

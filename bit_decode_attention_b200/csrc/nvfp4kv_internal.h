@@ -1,0 +1,59 @@
+// nvfp4kv_internal.h -- host-side declarations shared by the .cu files of
+// libnvfp4kv.so (launchers behind the C ABI in include/nvfp4kv.h).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/nvfp4kv.h"
+
+namespace nvfp4kv {
+
+// tokens per pipeline stage of the decode-attention kernel
+constexpr int kTile = 32;
+// sequences handled by one decode-attention launch
+constexpr int kMaxBatchPerLaunch = 512;
+// resident decode-attention CTAs per SM (the kernel is written for this)
+constexpr int kCtasPerSm = 2;
+
+int device_sm_count();  // multiprocessor count of the current device (cached)
+
+cudaError_t launch_calib(const void* x, bool f32, int64_t n, float* d_s_tensor, int32_t* d_status,
+                         cudaStream_t stream);
+
+cudaError_t launch_quantize_append(const void* x_new, bool f32, int n_new,
+                                   const int32_t* d_start_pos, int32_t* d_new_lens,
+                                   const float* d_s_tensor, const nvfp4_kv_plane& plane,
+                                   int32_t* d_status, cudaStream_t stream);
+
+cudaError_t launch_dequant_fp8(const nvfp4_kv_plane& plane, const float* d_s_tensor,
+                               const int32_t* d_seq_lens, uint8_t* out, int32_t* d_status,
+                               cudaStream_t stream);
+
+struct AttnLaunch {
+    const void* q;
+    bool q_f32;
+    int B, Hq, Hkv, S_max, D;
+    const uint8_t *kc, *ks, *vc, *vs;
+    const float *st_k, *st_v;
+    const int32_t* seq_lens;
+    float softmax_scale;
+    float* out;
+    float* partials;     // [2 * grid][g][D + 2]
+    int32_t* counters;   // [B * Hkv], zero between calls
+    int32_t* status;
+    int grid;            // CTAs
+};
+
+cudaError_t launch_decode_attention(const AttnLaunch& a, cudaStream_t stream);
+
+// workspace layout of nvfp4_decode_attention for one shape
+struct AttnWorkspace {
+    size_t counters_bytes;  // B * H_kv int32, padded to 256 bytes
+    size_t partial_floats;  // 2 * grid * g * (D + 2)
+    size_t total_bytes;
+    int grid;
+};
+AttnWorkspace attention_workspace(int B, int Hq, int Hkv, int D);
+
+}  // namespace nvfp4kv

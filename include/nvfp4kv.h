@@ -1,0 +1,181 @@
+/*
+ * nvfp4kv.h -- C ABI of libnvfp4kv.so: an NVFP4 KV cache with fused
+ * NVFP4 -> FP8 decode attention for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (sources are web pages, cited by title/section):
+ *
+ *   [NVFP4-KV] "NVIDIA解説: NVFP4 KV Cacheで長コンテキストLLM推論を最適化 --
+ *              メモリ50%削減・TTFT 3倍高速化" (0h-n0.github.io; a summary of
+ *              NVIDIA's technical blog on the NVFP4 KV cache).
+ *   [rc17]     "TensorRT-LLM rc17 が SM121（DGX Spark）向けに NVFP4 MoE
+ *              バックエンドと NVFP4 KV キャッシュを追加".
+ *   [FR-lesson] "Compilation d'inferences spécialisées en matériel FP8 et
+ *              NVFP4 sur Blackwell".
+ *
+ *   Storage ([NVFP4-KV] "E2M1 + 2レベルスケーリング"): every K or V element
+ *   is an E2M1 code (sign 1, exponent 2, mantissa 1; values 0, 0.5, 1, 1.5,
+ *   2, 3, 4, 6 and negatives), every 16 consecutive elements along head_dim
+ *   share one E4M3 scale byte s_block, and the whole tensor shares one fp32
+ *   scale s_tensor:  x ~ x_q * s_block * s_tensor.
+ *   Flow ([NVFP4-KV] "量子化・逆量子化フロー", [rc17] "物語の KV キャッシュ側"):
+ *   new tokens are quantized on append; at attention time the cache is
+ *   dequantized to FP8 and FP8 attention runs with an FP32 accumulator
+ *   ([FR-lesson] "Le type de Blackwell").
+ *
+ * Exact arithmetic (where the pages are silent, these are the readings):
+ *   s_tensor = fl32(amax / 2688)          (2688 = 6 * 448; amax == 0 -> 1)
+ *   d6       = fl32(6 * s_tensor)
+ *   s_block  = E4M3(fl32(amax_blk / d6))  (round to nearest even, satfinite)
+ *   den      = fl32(value(s_block) * s_tensor)
+ *   code_i   = E2M1(fl32(x_i / den))      (nearest, ties to even code,
+ *                                          saturating; sign copied, so a
+ *                                          negative value rounding to zero
+ *                                          gives code 0x8; den == 0 gives
+ *                                          signed-zero codes)
+ *   fp8_i    = E4M3(fl32(fl32(|code_i| * value(s_block)) * s_tensor)) with
+ *              the code's sign as the FP8 sign bit
+ *   out[b][h] = softmax(q[b][h] . K^T * softmax_scale) . V over the first
+ *              seq_lens[b] tokens of KV head h / (H_q / H_kv), using the FP8
+ *              values of K and V; an empty sequence gives a zero row.
+ *
+ * Memory layout of one cache plane (K or V; caller-owned device memory):
+ *   codes  : uint8 [B][H_kv][S_max][D/2]; byte j of a token row holds
+ *            element 2j in its low nibble and element 2j+1 in its high nibble
+ *   scales : uint8 [B][H_kv][S_max][D/16]; byte j scales elements 16j..16j+15
+ *   Both pointers 16-byte aligned; S_max a multiple of 16; D in {64, 128}.
+ *
+ * Conventions for every call:
+ *   - All pointers named d_* or described as device memory are CUDA device
+ *     pointers on the current device; plane structs and sizes are host data.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream) and
+ *     allocate nothing.  The return value reports host-side validation and
+ *     launch errors only.
+ *   - Conditions found on the device (a sequence past S_max, a non-finite
+ *     or non-positive tensor scale, a pipeline wait that gave up) are written
+ *     to *d_status (int32, device memory, may be NULL): the first error code
+ *     is kept (compare-and-swap from 0); the caller zeroes it.
+ *   - No call aborts, traps or throws.
+ */
+#ifndef NVFP4KV_H
+#define NVFP4KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* nvfp4_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or shape */
+    NVFP4_ERR_UNSUPPORTED = 2,  /* valid request this build does not handle */
+    NVFP4_ERR_CAPACITY = 3,     /* a sequence would pass S_max */
+    NVFP4_ERR_NONFINITE = 4,    /* non-finite data or tensor scale */
+    NVFP4_ERR_CUDA = 5,         /* a CUDA runtime call failed */
+    NVFP4_ERR_TIMEOUT = 6,      /* a bounded device-side wait gave up */
+    NVFP4_ERR_WORKSPACE = 7     /* workspace missing or too small */
+} nvfp4_status;
+
+typedef enum {
+    NVFP4_IN_BF16 = 0,          /* bfloat16 inputs */
+    NVFP4_IN_F32 = 1            /* float32 inputs */
+} nvfp4_dtype;
+
+/* One NVFP4 cache plane (K or V).  The struct lives in host memory; the
+ * two arrays it points to live in device memory (layout above). */
+typedef struct {
+    uint8_t* codes;   /* [B][H_kv][S_max][D/2] */
+    uint8_t* scales;  /* [B][H_kv][S_max][D/16] */
+    int32_t B;        /* sequences */
+    int32_t H_kv;     /* KV heads */
+    int32_t S_max;    /* token capacity per sequence, multiple of 16 */
+    int32_t D;        /* head_dim, 64 or 128 */
+} nvfp4_kv_plane;
+
+/* Human-readable name of a status value (static string). */
+const char* nvfp4_status_string(int status);
+
+/* Library version string (static). */
+const char* nvfp4_version(void);
+
+/* Bytes of ONE plane (codes + scales) for the given shape: B * H_kv * S_max *
+ * (D/2 + D/16).  Per element that is 4 code bits plus 8/16 scale bits = 4.5
+ * bits, the format behind the memory table in [NVFP4-KV] "メモリ削減効果"
+ * (3.5x smaller than FP16, about 1.8x smaller than FP8).  Returns 0 for
+ * invalid shapes.  Host-only; needs no GPU. */
+size_t nvfp4_cache_bytes(int B, int H_kv, int S_max, int D);
+
+/* Calibrate the per-tensor scale ([NVFP4-KV] "E2M1 + 2レベルスケーリング",
+ * level 2: one FP32 scale per tensor).
+ *   x          device, n elements of `dtype` (any alignment)
+ *   d_s_tensor device float, written with fl32(amax / 2688), or 1.0 when
+ *              amax == 0.  If any element is Inf/NaN, *d_s_tensor is set to
+ *              NaN and NVFP4_ERR_NONFINITE goes to *d_status.
+ * Launches a 4-byte memset and two kernels on `stream`.  n == 0 gives 1.0. */
+nvfp4_status nvfp4_calib_tensor_scale(const void* x, nvfp4_dtype dtype, int64_t n,
+                                      float* d_s_tensor, int32_t* d_status,
+                                      nvfp4_stream_t stream);
+
+/* Quantize n_new tokens per sequence and append them to a plane
+ * ([NVFP4-KV] "量子化・逆量子化フロー": new K/V are quantized to NVFP4 in
+ * 16-element blocks and stored in the cache).
+ *   x_new        device [B][n_new][H_kv][D] of `dtype`, 16-byte aligned
+ *   d_start_pos  device int32 [B]: tokens go to slots start..start+n_new-1
+ *   d_new_lens   device int32 [B] or NULL: written with start + n_new; must
+ *                not alias d_start_pos
+ *   d_s_tensor   device float, the tensor scale from calibration (> 0)
+ *   plane        host struct describing the destination plane
+ * A sequence with start < 0 or start + n_new > S_max is skipped entirely and
+ * NVFP4_ERR_CAPACITY goes to *d_status; a non-finite or non-positive tensor
+ * scale skips everything with NVFP4_ERR_NONFINITE.  n_new == 0 is a no-op. */
+nvfp4_status nvfp4_kv_quantize_append(const void* x_new, nvfp4_dtype dtype, int n_new,
+                                      const int32_t* d_start_pos, int32_t* d_new_lens,
+                                      const float* d_s_tensor, const nvfp4_kv_plane* plane,
+                                      int32_t* d_status, nvfp4_stream_t stream);
+
+/* Dequantize a plane to FP8 E4M3 bytes ([NVFP4-KV] "量子化・逆量子化フロー":
+ * NVFP4 -> FP8 before attention).
+ *   d_seq_lens device int32 [B]; only slots t < seq_lens[b] are written
+ *   out_e4m3   device uint8 [B][H_kv][S_max][D], 16-byte aligned
+ * Lengths past S_max are clamped and reported as NVFP4_ERR_CAPACITY. */
+nvfp4_status nvfp4_kv_dequant_fp8(const nvfp4_kv_plane* plane, const float* d_s_tensor,
+                                  const int32_t* d_seq_lens, uint8_t* out_e4m3,
+                                  int32_t* d_status, nvfp4_stream_t stream);
+
+/* Workspace bytes nvfp4_decode_attention needs on the current device for
+ * this shape (split-K partial results and per-(sequence, KV head) arrival
+ * counters).  Returns 0 for invalid shapes.  The workspace must be
+ * zero-filled once after allocation; every completed call leaves its
+ * counters at zero again, so it can be reused without clearing.  Calls that
+ * share one workspace must not overlap on the GPU. */
+size_t nvfp4_decode_attention_workspace(int B, int H_q, int H_kv, int D);
+
+/* Decode attention over an NVFP4 cache with FP8 dequantization fused in
+ * ([NVFP4-KV] "量子化・逆量子化フロー": FP8 attention and the context matmul
+ * on the dequantized cache; [FR-lesson] "Le type de Blackwell": FP32
+ * accumulator).  One query token per sequence, grouped-query attention.
+ *   q            device [B][H_q][D] of `q_dtype`, 16-byte aligned
+ *   H_q          query heads; H_q % H_kv == 0 and H_q / H_kv <= 16
+ *   k, v         host structs of the K and V planes (same B, H_kv, S_max, D)
+ *   d_s_tensor_k, d_s_tensor_v  device floats
+ *   d_seq_lens   device int32 [B], tokens to attend per sequence (<= S_max)
+ *   softmax_scale  0 selects 1/sqrt(D)
+ *   out          device float [B][H_q][D]
+ *   workspace    device, >= nvfp4_decode_attention_workspace(...) bytes,
+ *                zero-filled once (see above), 16-byte aligned
+ * Lengths past S_max are clamped and reported as NVFP4_ERR_CAPACITY.
+ * Batches larger than 1024 sequences are processed in launches of 1024. */
+nvfp4_status nvfp4_decode_attention(const void* q, nvfp4_dtype q_dtype, int H_q,
+                                    const nvfp4_kv_plane* k, const nvfp4_kv_plane* v,
+                                    const float* d_s_tensor_k, const float* d_s_tensor_v,
+                                    const int32_t* d_seq_lens, float softmax_scale,
+                                    float* out, void* workspace, size_t workspace_bytes,
+                                    int32_t* d_status, nvfp4_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4KV_H */

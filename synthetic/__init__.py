@@ -153,3 +153,31 @@ def capacity(max_len: int, extra: int = 0) -> int:
     """Cache capacity S_max for a workload: max_len + extra rounded up to 16."""
     n = max_len + extra
     return (n + 15) // 16 * 16
+
+
+def random_planes(seed: int, B: int, H_kv: int, S_max: int, D: int, max_scale_byte: int = 0x7E):
+    """Uniformly random NVFP4 planes (every code nibble, scale bytes 0..max),
+    uint8 tensors [B][H_kv][S_max][D/2] and [B][H_kv][S_max][D/16]."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    codes = torch.randint(0, 256, (B, H_kv, S_max, D // 2), generator=g, dtype=torch.int32)
+    scales = torch.randint(0, max_scale_byte + 1, (B, H_kv, S_max, D // 16), generator=g,
+                           dtype=torch.int32)
+    return codes.to(torch.uint8), scales.to(torch.uint8)
+
+
+def special_blocks(D: int = 128) -> torch.Tensor:
+    """A handful of hand-picked token rows [n][D] that hit the corner cases of
+    block quantization: all-zero and signed-zero blocks, one-hot blocks, exact
+    grid midpoints, tiny values, and values far beyond the calibrated range."""
+    rows = []
+    z = torch.zeros(D)
+    rows.append(z.clone())
+    r = z.clone(); r[1::2] = -0.0; rows.append(r)
+    r = z.clone(); r[0] = 1.0; r[17] = -3.0; rows.append(r)
+    r = torch.tensor([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0] * (D // 8)); rows.append(r)
+    r = torch.tensor([-0.25, 0.5, -1.0, 1.5, -2.0, 3.0, -4.0, 6.0] * (D // 8)); rows.append(r)
+    r = torch.full((D,), 1e-30); r[::3] = -2e-38; rows.append(r)
+    r = torch.linspace(-50.0, 50.0, D); rows.append(r)
+    r = torch.linspace(-1e4, 3e4, D); rows.append(r)
+    return torch.stack(rows)

@@ -1,0 +1,102 @@
+"""The C-ABI library loads, exports every symbol include/*.h declares, and its
+host-only logic (sizes, argument validation) behaves as documented.  No
+kernel is launched here: every call below returns before reaching the GPU.
+"""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import oracle
+from bit_decode_attention_b200 import _native
+from bit_decode_attention_b200 import build as native_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    native_build.build()
+    return _native.lib()
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(nvfp4_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_native.EXPORTS)
+
+
+def test_version_and_status_strings(lib):
+    assert b"sm_100a" in lib.nvfp4_version()
+    assert lib.nvfp4_status_string(0) == b"ok"
+    assert lib.nvfp4_status_string(3) == b"sequence past cache capacity"
+    assert lib.nvfp4_status_string(99) == b"unknown status"
+
+
+def test_cache_bytes_matches_oracle_memory_model(lib):
+    # one plane = B*H*S*D elements at 4.5 bits; K and V together follow the
+    # KV-memory formula of the pages with 4.5-bit elements
+    for B, H, S, D in [(8, 8, 4096, 128), (1, 8, 65536, 128), (3, 2, 48, 64)]:
+        plane = lib.nvfp4_cache_bytes(B, H, S, D)
+        assert plane == B * H * S * (D // 2 + D // 16)
+        assert 2 * plane == oracle.kv_bytes(1, H, D, S, B, oracle.nvfp4_bits_per_element())
+    assert lib.nvfp4_cache_bytes(1, 0, 16, 128) == 0
+    assert lib.nvfp4_cache_bytes(1, 1, 16, 40) == 0
+
+
+def test_workspace_size(lib):
+    assert lib.nvfp4_decode_attention_workspace(8, 32, 8, 128) > 0
+    assert lib.nvfp4_decode_attention_workspace(8, 30, 8, 128) == 0   # H_q % H_kv
+    assert lib.nvfp4_decode_attention_workspace(8, 8 * 17, 8, 128) == 0  # group > 16
+    assert lib.nvfp4_decode_attention_workspace(8, 32, 8, 96) == 0     # head_dim
+
+
+def _plane(B=1, H=1, S=16, D=128, codes=16, scales=16):
+    return _native.KVPlaneStruct(codes, scales, B, H, S, D)
+
+
+def test_argument_validation_without_gpu(lib):
+    p = _plane()
+    bad_s = _plane(S=24)
+    bad_d = _plane(D=96)
+    misaligned = _plane(codes=17)
+    dev = ctypes.c_void_p(64)  # never dereferenced: every call below fails validation
+    INVALID, WS = _native.NVFP4_ERR_INVALID_ARG, _native.NVFP4_ERR_WORKSPACE
+    qa = lib.nvfp4_kv_quantize_append
+    assert qa(dev, 0, 1, dev, None, dev, ctypes.byref(bad_s), None, None) == INVALID
+    assert qa(dev, 0, 1, dev, None, dev, ctypes.byref(bad_d), None, None) == INVALID
+    assert qa(dev, 0, 1, dev, None, dev, ctypes.byref(misaligned), None, None) == INVALID
+    assert qa(dev, 7, 1, dev, None, dev, ctypes.byref(p), None, None) == INVALID   # dtype
+    assert qa(dev, 0, 1, dev, dev, dev, ctypes.byref(p), None, None) == INVALID    # aliasing
+    assert qa(ctypes.c_void_p(72), 0, 1, dev, None, dev, ctypes.byref(p), None, None) == INVALID
+    assert qa(dev, 0, 0, dev, None, dev, ctypes.byref(p), None, None) == 0         # no-op
+    dq = lib.nvfp4_kv_dequant_fp8
+    assert dq(ctypes.byref(p), None, dev, dev, None, None) == INVALID
+    assert dq(ctypes.byref(p), dev, dev, ctypes.c_void_p(65), None, None) == INVALID
+    at = lib.nvfp4_decode_attention
+    k, v = _plane(B=2, H=2), _plane(B=2, H=2)
+    v_other = _plane(B=2, H=2, S=32)
+    args = lambda hq, kk, vv, ws, nbytes: (dev, 0, hq, ctypes.byref(kk), ctypes.byref(vv), dev, dev,
+                                           dev, ctypes.c_float(0.0), dev, ws, nbytes, None, None)
+    assert at(*args(3, k, v, dev, 1 << 30)) == INVALID            # H_q % H_kv
+    assert at(*args(4, k, v_other, dev, 1 << 30)) == INVALID      # planes disagree
+    assert at(*args(2 * 17, k, v, dev, 1 << 30)) == _native.NVFP4_ERR_UNSUPPORTED
+    assert at(*args(4, k, v, None, 0)) == WS
+    assert at(*args(4, k, v, dev, 16)) == WS
+    cal = lib.nvfp4_calib_tensor_scale
+    assert cal(dev, 0, -1, dev, None, None) == INVALID
+    assert cal(dev, 0, 10, None, None, None) == INVALID
+    assert cal(ctypes.c_void_p(65), 0, 10, dev, None, None) == INVALID   # bf16 misaligned

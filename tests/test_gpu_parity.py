@@ -1,0 +1,223 @@
+"""GPU parity: every kernel, called through the C-ABI binding, against the CPU
+oracle on the same seeded inputs.  Bit-exact for the tensor scale, packed
+codes, scale bytes and FP8 bytes; attention within max-abs 2e-2 and
+mean-abs 2e-3 of the fp64 oracle over the same FP8 values.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from cases import Case, assert_attention_close, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nv():
+    import bit_decode_attention_b200 as nv
+    return nv
+
+
+# ---------------------------------------------------------------------------
+# calibration
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("n", [1, 7, 1000, (1 << 20) + 3])
+def test_calib_bit_exact(nv, dtype, n):
+    w = synthetic.shrink(synthetic.get("long64k"), dtype=dtype)
+    x = synthetic.kv_tokens(w, (n + 1023) // 1024, "k").reshape(-1)[:n]
+    for offset in (0, 1):       # aligned and misaligned base pointer
+        xs = x[offset:] if n > 1 else x
+        st, want = oracle.tensor_scale(xs.numpy())
+        dev = to_dev(x, dtype)[offset:] if n > 1 else to_dev(x, dtype)
+        got = nv.nvfp4_calib_tensor_scale(dev).item()
+        assert st == 0
+        assert np.float32(got).view(np.uint32) == np.float32(want).view(np.uint32)
+
+
+def test_calib_zero_and_nonfinite(nv):
+    z = torch.zeros(100, device="cuda", dtype=torch.bfloat16)
+    assert nv.nvfp4_calib_tensor_scale(z).item() == 1.0
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    x = torch.ones(100, device="cuda")
+    x[37] = float("nan")
+    s = nv.nvfp4_calib_tensor_scale(x, status=status)
+    assert np.isnan(s.item()) and status.item() == nv.NVFP4_ERR_NONFINITE
+    st_o, _ = oracle.tensor_scale(x.cpu().numpy())
+    assert st_o == 4
+
+
+# ---------------------------------------------------------------------------
+# quantize + append, dequant
+# ---------------------------------------------------------------------------
+def _check_planes(case, batch_indices=None):
+    bs = list(range(case.w.B)) if batch_indices is None else list(batch_indices)
+    for b in bs:
+        kc, ks, vc, vs = case.oracle_planes(b)
+        L = case.lens[b]
+        np.testing.assert_array_equal(case.k.codes[b, :, :L].cpu().numpy(), kc[0, :, :L])
+        np.testing.assert_array_equal(case.k.scales[b, :, :L].cpu().numpy(), ks[0, :, :L])
+        np.testing.assert_array_equal(case.v.codes[b, :, :L].cpu().numpy(), vc[0, :, :L])
+        np.testing.assert_array_equal(case.v.scales[b, :, :L].cpu().numpy(), vs[0, :, :L])
+
+
+SMALL_CASES = {
+    "tiny": lambda: Case(synthetic.get("tiny")),
+    "gqa_ragged": lambda: Case(synthetic.shrink(synthetic.get("gqa"), B=4), lens=[4097, 1, 33, 640]),
+    "long_outliers": lambda: Case(synthetic.shrink(synthetic.get("long64k"), L=20000)),
+    "ragged16": lambda: Case(synthetic.shrink(synthetic.get("ragged"), B=16)),
+    "moe_g12_chunked": lambda: Case(synthetic.shrink(synthetic.get("moe128k"), L=5000),
+                                    prefill_chunk=2048),
+}
+
+
+@pytest.fixture(scope="module", params=list(SMALL_CASES))
+def case(request):
+    c = SMALL_CASES[request.param]()
+    assert c.status.item() == 0
+    return c
+
+
+def test_tensor_scale_matches(case):
+    for dev, want in ((case.sk, case.sk_o), (case.sv, case.sv_o)):
+        assert np.float32(dev.item()).view(np.uint32) == np.float32(want).view(np.uint32)
+
+
+def test_quantize_append_bit_exact(case):
+    _check_planes(case)
+
+
+def test_dequant_fp8_bit_exact(nv, case):
+    out = nv.nvfp4_kv_dequant_fp8(case.k, case.sk, case.seq_lens).cpu().numpy()
+    kc, ks, vc, vs = case.oracle_planes()
+    want = oracle.dequant_planes(kc, ks, case.sk_o, np.array(case.lens, np.int32))
+    for b, L in enumerate(case.lens):
+        np.testing.assert_array_equal(out[b, :, :L], want[b, :, :L])
+
+
+def test_attention_parity(case):
+    got = case.gpu_attention().cpu().numpy()
+    want = case.oracle_attention()
+    assert_attention_close(got, want)
+    assert case.status.item() == 0
+
+
+def test_special_blocks_bit_exact(nv):
+    rows = synthetic.special_blocks(128)
+    for dtype in ("f32", "bf16"):
+        x = rows.to(torch.bfloat16).float() if dtype == "bf16" else rows
+        x = x.view(1, rows.shape[0], 1, 128).contiguous()      # B=1, n tokens, H=1
+        for st in (np.float32(1.0), np.float32(0.01), np.float32(1e-30), np.float32(3e4)):
+            plane = nv.KVPlane.allocate(1, 1, 16, 128)
+            s = torch.tensor([st], device="cuda")
+            start = torch.zeros(1, dtype=torch.int32, device="cuda")
+            nv.nvfp4_kv_quantize_append(to_dev(x, dtype), start, s, plane)
+            kc, ks = oracle.new_planes(1, 1, 16, 128)
+            assert oracle.quantize_append(x.numpy(), np.zeros(1, np.int32), st, kc, ks) == 0
+            n = rows.shape[0]
+            np.testing.assert_array_equal(plane.codes[0, 0, :n].cpu().numpy(), kc[0, 0, :n])
+            np.testing.assert_array_equal(plane.scales[0, 0, :n].cpu().numpy(), ks[0, 0, :n])
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_dequant_random_planes_bit_exact(nv, D):
+    B, H, S = 2, 3, 64
+    codes, scales = synthetic.random_planes(7 + D, B, H, S, D)
+    plane = nv.KVPlane(codes.cuda(), scales.cuda())
+    lens = np.array([64, 37], np.int32)
+    for st in (1.0, 0.0371, 2.0 ** -20, 1e-8, 7.5):
+        s = torch.tensor([st], dtype=torch.float32, device="cuda")
+        got = nv.nvfp4_kv_dequant_fp8(plane, s, torch.from_numpy(lens).cuda()).cpu().numpy()
+        want = oracle.dequant_planes(codes.numpy(), scales.numpy(), np.float32(st), lens)
+        for b in range(B):
+            np.testing.assert_array_equal(got[b, :, :lens[b]], want[b, :, :lens[b]])
+
+
+def test_append_capacity_and_new_lens(nv):
+    w = synthetic.shrink(synthetic.get("gqa"), B=3, Hkv=2, Hq=4)
+    x = synthetic.kv_tokens(w, 5, "k")
+    plane = nv.KVPlane.allocate(3, 2, 16, 128)
+    s = torch.tensor([0.01], device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    start = torch.tensor([0, 12, 11], dtype=torch.int32, device="cuda")
+    new_lens = torch.full((3,), -7, dtype=torch.int32, device="cuda")
+    nv.nvfp4_kv_quantize_append(to_dev(x, "bf16"), start, s, plane, new_lens=new_lens, status=status)
+    assert status.item() == nv.NVFP4_ERR_CAPACITY
+    assert new_lens.tolist() == [5, -7, 16]
+    assert not plane.codes[1].any().item()
+    kc, ks = oracle.new_planes(3, 2, 16, 128)
+    assert oracle.quantize_append(x.numpy(), start.cpu().numpy(), np.float32(0.01), kc, ks) == 3
+    np.testing.assert_array_equal(plane.codes.cpu().numpy(), kc)
+    np.testing.assert_array_equal(plane.scales.cpu().numpy(), ks)
+
+
+def test_bad_tensor_scale_reports(nv):
+    plane = nv.KVPlane.allocate(1, 1, 16, 64)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    x = torch.ones(1, 1, 1, 64, device="cuda")
+    for bad in (0.0, -1.0, float("inf"), float("nan")):
+        status.zero_()
+        nv.nvfp4_kv_quantize_append(x, torch.zeros(1, dtype=torch.int32, device="cuda"),
+                                    torch.tensor([bad], device="cuda"), plane, status=status)
+        assert status.item() == nv.NVFP4_ERR_NONFINITE
+    assert not plane.codes.any().item()
+
+
+# ---------------------------------------------------------------------------
+# attention edge cases
+# ---------------------------------------------------------------------------
+def test_attention_empty_and_short_sequences(nv):
+    c = Case(synthetic.shrink(synthetic.get("gqa"), B=5, Hq=8, Hkv=2), lens=[0, 5, 0, 1, 31])
+    got = c.gpu_attention().cpu().numpy()
+    assert not got[0].any() and not got[2].any()
+    assert_attention_close(got, c.oracle_attention())
+
+
+def test_attention_q_dtypes_and_scale(nv):
+    c = Case(synthetic.shrink(synthetic.get("gqa"), B=2, Hq=16, Hkv=2, D=64), lens=[300, 77],
+             q_dtype="f32")
+    assert_attention_close(c.gpu_attention().cpu().numpy(), c.oracle_attention())
+    assert_attention_close(c.gpu_attention(softmax_scale=0.05).cpu().numpy(),
+                           c.oracle_attention(softmax_scale=0.05))
+    c2 = Case(synthetic.shrink(synthetic.get("tiny"), B=2, Hq=4, Hkv=1, dtype="bf16"), lens=[256, 40])
+    assert_attention_close(c2.gpu_attention().cpu().numpy(), c2.oracle_attention())
+
+
+def test_attention_fewer_tiles_than_ctas(nv):
+    # one unit spread over CTAs with empty ranges in between (94 tiles < grid)
+    c = Case(synthetic.shrink(synthetic.get("long64k"), Hq=2, Hkv=1, L=3000))
+    assert_attention_close(c.gpu_attention().cpu().numpy(), c.oracle_attention())
+
+
+def test_attention_group_sizes(nv):
+    for g in (1, 2, 3, 8, 12, 16):
+        c = Case(synthetic.shrink(synthetic.get("gqa"), B=2, Hq=2 * g, Hkv=2), lens=[700, 129])
+        assert_attention_close(c.gpu_attention().cpu().numpy(), c.oracle_attention())
+
+
+def test_attention_large_batch_is_chunked(nv):
+    w = synthetic.shrink(synthetic.get("ragged"), B=600, Hq=2, Hkv=1, L_range=(1, 40))
+    c = Case(w)
+    assert_attention_close(c.gpu_attention().cpu().numpy(), c.oracle_attention())
+
+
+def test_attention_workspace_reuse_and_repeatability(nv):
+    c = Case(synthetic.shrink(synthetic.get("long64k"), L=9000))
+    ws = nv.new_workspace(1, 64, 8, 128)
+    a = c.gpu_attention(workspace=ws).cpu()
+    b = c.gpu_attention(workspace=ws).cpu()
+    assert torch.equal(a, b)
+    counters = ws[: 8 * 4].view(torch.int32)
+    assert not counters.any().item()      # arrival counters are left at zero
+
+
+def test_attention_length_past_capacity_reports(nv):
+    c = Case(synthetic.shrink(synthetic.get("gqa"), B=2, Hq=8, Hkv=2), lens=[40, 16])
+    bad = torch.tensor([40, c.S_max + 5], dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = nv.nvfp4_decode_attention(c.q_dev, c.k, c.v, c.sk, c.sv, bad, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == nv.NVFP4_ERR_CAPACITY
+    assert torch.isfinite(out).all().item()
