@@ -281,7 +281,7 @@ def run_steps(graph_full, graph_tail, per_graph, n_steps):
         graph_tail[n_steps % per_graph].replay()
 
 
-def time_decode(wl, steps, warmup, world, sampler=None, graph_steps=None):
+def time_decode(wl, steps, warmup, world, sampler=None, graph_steps=None, nvtx_name="timed"):
     """Returns (elapsed_ms max over ranks, attention ms per launch, clocks)."""
     G = graph_steps or wl.R * max(1, 16 // wl.R)
     G = max(G, wl.R)
@@ -296,18 +296,16 @@ def time_decode(wl, steps, warmup, world, sampler=None, graph_steps=None):
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_wall0 = time.time()
+    torch.cuda.nvtx.range_push(nvtx_name)
     start.record()
     run_steps(full, tails, G, steps)
     end.record()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     t_wall1 = time.time()
     if world > 1:
         torch.distributed.barrier()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = t.item()
+    ms = max_over_ranks(start.elapsed_time(end), world, "cuda")
     # the attention launches of the last full replay inside the timed region
     att = [a.elapsed_time(b) for a, b in evs] if steps >= G else []
     clocks = sampler.summary(t_wall0, t_wall1) if sampler is not None else None
@@ -465,6 +463,20 @@ def config_block(w, L0, wl):
 
 
 # ---------------------------------------------------------------------------
+def max_over_ranks(value, world, device):
+    """The largest per-rank value (elapsed time) across the process group."""
+    if world <= 1:
+        return value
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.item()
+
+
+def job_throughput(world, tokens_per_step, steps, max_ms):
+    """Whole-job KV-tokens/s: the tokens all ranks processed over the slowest rank's time."""
+    return world * tokens_per_step * steps / (max_ms / 1e3)
+
+
 def replicas_for(bytes_per_replica, l2_bytes):
     return max(2, math.ceil(2 * l2_bytes / bytes_per_replica))
 
@@ -509,7 +521,7 @@ def main():
     status = wl.status.item()
 
     tokens = wl.tokens_per_step()
-    value = world * tokens * args.steps / (ms / 1e3)
+    value = job_throughput(world, tokens, args.steps, ms)
     peak, peak_kind = measured_peaks()
     roof = None
     if att_ms:
@@ -546,7 +558,7 @@ def main():
         per = lw.B * lw.L * kv_bytes_per_token(lw.Hkv, lw.D)
         lwl = DecodeWorkload(lw, lw.L, replicas_for(per, l2), with_append=False)
         n_aux = max(64, min(2000, args.steps))
-        lms, latt, lat_n, _ = time_decode(lwl, n_aux, 20, world)
+        lms, latt, lat_n, _ = time_decode(lwl, n_aux, 20, world, nvtx_name="timed_aux")
         ach = lwl.attention_bytes() / (latt / 1e3) / 1e9 if latt else None
         aux["long64k_attention"] = {
             "workload": "long64k: B1 Hq64 Hkv8 D128 L65536, decode attention only (split-K)",

@@ -68,6 +68,14 @@ struct Geometry {
     static_assert(STAGE % 16 == 0, "stage must keep 16-byte alignment");
 };
 
+// scratch of the split-K merge (see combine_partials)
+struct CombineSmem {
+    int32_t slot[32];         // partial slot of chunk contributor j, -1 if none
+    float w[16][32];          // weight of contributor j for query q
+    float M[16];
+    float l[16];
+};
+
 template <int D, int NT>
 struct __align__(16) Smem {
     static constexpr int kStages = Ring<NT>::kStages;
@@ -80,6 +88,7 @@ struct __align__(16) Smem {
     int32_t prefix[kMaxBatchPerLaunch + 1];
     float merge_m[kWarps][8 * NT];
     float merge_l[kWarps][8 * NT];
+    CombineSmem comb;
     int32_t warp_tot[kWarps];
     int32_t last_flag;
 };
@@ -197,17 +206,41 @@ __device__ __forceinline__ uint32_t pow2_bits(int e) {  // 2^e as fp32 bits, e i
     return (uint32_t)(127 + e) << 23;
 }
 
-// Load the query fragments of unit (b, h) for this lane.  Lane (gid, tig)
-// holds query row j = 8*nt + gid, elements [EK*tig, EK*tig + EK) as f16
-// pairs in natural order: qf[s][nt][0] = elements (4s, 4s+1),
-// qf[s][nt][1] = (4s+2, 4s+3) -- the same order the K fragments use.
-// Each row is scaled by 2^e so that its largest |q| lands below 2^14;
-// cscale[nt][c] = softmax_scale * log2(e) * 2^-e of the row in column
+// ---------------------------------------------------------------------------
+// Query operands.  Lane (gid, tig) holds query row j = 8*nt + gid, head_dim
+// elements [EK*tig, EK*tig + EK): the same elements its K fragments carry,
+// in the same order, so the contraction runs over a permutation of head_dim
+// that both operands share.
+//
+//  * bf16 queries -> FP8 (E4M3) MMA operands: every bf16 value (8 significant
+//    bits) is split exactly into hi = E4M3(q') and lo = E4M3((q' - hi) * 16),
+//    q' = q * 2^e with e chosen per row so that max |q'| < 256.  The two
+//    products go to separate accumulators: s = s_hi + s_lo / 16.
+//  * fp32 queries -> f16 MMA operands: hi = f16(q'), lo = f16(q' - hi)
+//    (22 bits), q' scaled so that max |q'| < 2^14; both accumulate together.
+// cscale[nt][c] = softmax_scale * log2(e) * 2^-e of the row in score column
 // 2*tig + c.
+// ---------------------------------------------------------------------------
+template <int D, int NT, bool QF32>
+struct QueryFrags;
+
+template <int D, int NT>
+struct QueryFrags<D, NT, false> {
+    static constexpr int S = D / 32;          // k32 steps
+    uint32_t hi[S][NT][2], lo[S][NT][2];
+    float cscale[NT][2];
+};
+
+template <int D, int NT>
+struct QueryFrags<D, NT, true> {
+    static constexpr int S = D / 16;          // k16 steps
+    uint32_t hi[S][NT][2], lo[S][NT][2];
+    float cscale[NT][2];
+};
+
 template <int D, int NT, bool QF32>
 __device__ __forceinline__ void load_q(const Params& p, int b, int h, int gid, int tig,
-                                       uint32_t (&qf)[D / 16][NT][2], uint32_t (&ql)[D / 16][NT][2],
-                                       float (&cscale)[NT][2]) {
+                                       QueryFrags<D, NT, QF32>& qf) {
     using G = Geometry<D>;
     const float base = p.softmax_scale * kLog2e;
 #pragma unroll
@@ -216,7 +249,7 @@ __device__ __forceinline__ void load_q(const Params& p, int b, int h, int gid, i
         const bool valid = j < p.g;
         float v[G::EK];
         const int64_t row = ((int64_t)b * p.Hq + (int64_t)h * p.g + (valid ? j : 0)) * D + G::EK * tig;
-        if (QF32) {
+        if constexpr (QF32) {
             const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.q) + row);
 #pragma unroll
             for (int i = 0; i < G::EK / 4; ++i) {
@@ -241,31 +274,190 @@ __device__ __forceinline__ void load_q(const Params& p, int b, int h, int gid, i
         for (int i = 0; i < G::EK; ++i) amax = fmaxf(amax, fabsf(v[i]));
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+        constexpr int kTopExp = QF32 ? 14 : 8;   // max |q'| < 2^kTopExp
         int e = 0;
         if (amax > 0.0f && amax <= 3.4028234663852886e38f) {
             int ex;
-            frexpf(amax, &ex);                 // amax < 2^ex
-            e = 14 - ex;
+            frexpf(amax, &ex);                    // amax < 2^ex
+            e = kTopExp - ex;
             e = e < -126 ? -126 : (e > 126 ? 126 : e);
         }
         const float up = __uint_as_float(pow2_bits(e));
         const float down = __uint_as_float(pow2_bits(-e));
 #pragma unroll
-        for (int s = 0; s < G::KS; ++s) {
+        for (int i = 0; i < G::EK; ++i) v[i] *= up;
+        if constexpr (QF32) {
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const float x0 = v[4 * s + 2 * k] * up, x1 = v[4 * s + 2 * k + 1] * up;
-                const uint32_t hi = pack_f16x2(x0, x1);
-                qf[s][nt][k] = hi;
-                if (QF32) ql[s][nt][k] = pack_f16x2(x0 - f16_lo_to_float(hi), x1 - f16_hi_to_float(hi));
+            for (int s = 0; s < G::KS; ++s) {
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const float x0 = v[4 * s + 2 * k], x1 = v[4 * s + 2 * k + 1];
+                    const uint32_t hi = pack_f16x2(x0, x1);
+                    qf.hi[s][nt][k] = hi;
+                    qf.lo[s][nt][k] = pack_f16x2(x0 - f16_lo_to_float(hi), x1 - f16_hi_to_float(hi));
+                }
+            }
+        } else {
+#pragma unroll
+            for (int s = 0; s < D / 32; ++s) {
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const float* x = v + 8 * s + 4 * k;
+                    const uint32_t h01 = e4m3x2_from_floats(x[0], x[1]);
+                    const uint32_t h23 = e4m3x2_from_floats(x[2], x[3]);
+                    uint32_t f01, f23;
+                    e4m3x4_to_f16x2x2(h01 | (h23 << 16), f01, f23);
+                    const uint32_t l01 = e4m3x2_from_floats((x[0] - f16_lo_to_float(f01)) * 16.0f,
+                                                            (x[1] - f16_hi_to_float(f01)) * 16.0f);
+                    const uint32_t l23 = e4m3x2_from_floats((x[2] - f16_lo_to_float(f23)) * 16.0f,
+                                                            (x[3] - f16_hi_to_float(f23)) * 16.0f);
+                    qf.hi[s][nt][k] = h01 | (h23 << 16);
+                    qf.lo[s][nt][k] = l01 | (l23 << 16);
+                }
             }
         }
-        // the score columns of this lane are query rows 2*tig and 2*tig+1 of n-tile nt,
-        // whose scale factors live in lanes (gid = 2*tig (+1), tig = 0)
+        // score column c of this lane is query row 2*tig + c; its scale lives
+        // in lanes (gid = 2*tig + c, tig = 0)
         const float f0 = __shfl_sync(0xFFFFFFFFu, down, (2 * tig) * 4);
         const float f1 = __shfl_sync(0xFFFFFFFFu, down, (2 * tig + 1) * 4);
-        cscale[nt][0] = base * f0;
-        cscale[nt][1] = base * f1;
+        qf.cscale[nt][0] = base * f0;
+        qf.cscale[nt][1] = base * f1;
+    }
+}
+
+// K operands of one 16-token sub-tile: lane (gid, tig) dequantizes tokens
+// gid and gid + 8, head_dim elements [EK*tig, EK*tig + EK) (EK/16 blocks).
+// fk[rr][w] = FP8 bytes of elements 4w .. 4w+3 of token gid + 8*rr.
+template <int D>
+__device__ __forceinline__ void dequant_k(const uint8_t* kc_s, const uint8_t* ks_s, const uint2* lut,
+                                          int sub, int gid, int tig, uint32_t (&fk)[2][D / 8]) {
+    using G = Geometry<D>;
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+        const int r = sub * 16 + gid + 8 * rr;
+        if constexpr (D == 128) {
+            const uint4 x = *reinterpret_cast<const uint4*>(kc_s + r * G::KB + 16 * tig);
+            const uint32_t sb = *reinterpret_cast<const uint16_t*>(ks_s + r * G::SB + 2 * tig);
+            const uint2 l0 = lut[sb & 0x7F];
+            const uint2 l1 = lut[(sb >> 8) & 0x7F];
+            dequant_word(x.x, l0.x, l0.y, fk[rr][0], fk[rr][1]);
+            dequant_word(x.y, l0.x, l0.y, fk[rr][2], fk[rr][3]);
+            dequant_word(x.z, l1.x, l1.y, fk[rr][4], fk[rr][5]);
+            dequant_word(x.w, l1.x, l1.y, fk[rr][6], fk[rr][7]);
+        } else {
+            const uint2 x = *reinterpret_cast<const uint2*>(kc_s + r * G::KB + 8 * tig);
+            const uint2 l0 = lut[ks_s[r * G::SB + tig] & 0x7F];
+            dequant_word(x.x, l0.x, l0.y, fk[rr][0], fk[rr][1]);
+            dequant_word(x.y, l0.x, l0.y, fk[rr][2], fk[rr][3]);
+        }
+    }
+}
+
+// V operands of one 16-token sub-tile: lane (gid, tig) dequantizes tokens
+// 2tig, 2tig+1, 2tig+8, 2tig+9 over channels [EV*gid, EV*gid + EV) (one
+// block); gv[tt][w] = FP8 bytes of channels 4w .. 4w+3 of token tt.
+template <int D>
+__device__ __forceinline__ void dequant_v(const uint8_t* vc_s, const uint8_t* vs_s, const uint2* lut,
+                                          int sub, int gid, int tig, uint32_t (&gv)[4][D / 32]) {
+    using G = Geometry<D>;
+#pragma unroll
+    for (int tt = 0; tt < 4; ++tt) {
+        const int r = sub * 16 + 2 * tig + (tt & 1) + 8 * (tt >> 1);
+        const uint2 l = lut[vs_s[r * G::SB + (G::EV * gid) / 16] & 0x7F];
+        if constexpr (D == 128) {
+            const uint2 x = *reinterpret_cast<const uint2*>(vc_s + r * G::KB + 8 * gid);
+            dequant_word(x.x, l.x, l.y, gv[tt][0], gv[tt][1]);
+            dequant_word(x.y, l.x, l.y, gv[tt][2], gv[tt][3]);
+        } else {
+            const uint32_t x = *reinterpret_cast<const uint32_t*>(vc_s + r * G::KB + 4 * gid);
+            dequant_word(x, l.x, l.y, gv[tt][0], gv[tt][1]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Split-K merge of one (sequence, KV head) unit by the last CTA to finish with
+// it.  The contributors are CTAs c_first..c_last (those with non-empty ranges);
+// each left (m, l, O) per query in its partial slot.  Out = sum_c w_c O_c /
+// sum_c w_c l_c with w_c = 2^(m_c - M), M = max_c m_c.  Contributors are
+// walked in chunks of 32 whose slot indices are computed once per chunk.
+// ---------------------------------------------------------------------------
+template <int D, int NT>
+__device__ __noinline__ void combine_partials(const Params& p, CombineSmem& cs, const Unit& u,
+                                                 int64_t T, int64_t N, int64_t c_first,
+                                                 int64_t c_last, int64_t slot_floats, int tid,
+                                                 int warp, int lane) {
+    constexpr int kThreads = kWarps * 32;
+    constexpr int kMaxOut = 8 * NT * D / kThreads;   // outputs per thread for g <= 8 * NT
+    const int g = p.g;
+    const int ncc = (int)(c_last - c_first + 1);
+    float acc[kMaxOut];
+#pragma unroll
+    for (int k = 0; k < kMaxOut; ++k) acc[k] = 0.0f;
+    for (int q = tid; q < g; q += kThreads) {
+        cs.M[q] = -INFINITY;
+        cs.l[q] = 0.0f;
+    }
+    for (int pass = 0; pass < 2; ++pass) {
+        for (int base = 0; base < ncc; base += 32) {
+            __syncthreads();
+            if (warp == 0) {
+                int sl = -1;
+                if (base + lane < ncc) {
+                    const int64_t cc = c_first + base + lane;
+                    if (range_start(cc, T, N) < range_start(cc + 1, T, N))
+                        sl = (int)partial_slot(cc, u.U0, T, N);
+                }
+                cs.slot[lane] = sl;
+            }
+            __syncthreads();
+            const int sl = cs.slot[lane];
+            for (int q = warp; q < g; q += kWarps) {
+                const float* part = p.partials + (int64_t)(sl < 0 ? 0 : sl) * slot_floats;
+                const float m = sl < 0 ? -INFINITY : __ldcg(part + g * D + q);
+                if (pass == 0) {
+                    float mx = m;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+                    if (lane == 0) cs.M[q] = fmaxf(cs.M[q], mx);
+                } else {
+                    const float M = cs.M[q];
+                    const float w = (m == -INFINITY) ? 0.0f : fast_exp2(m - M);
+                    cs.w[q][lane] = w;
+                    float lw = (w == 0.0f) ? 0.0f : w * __ldcg(part + g * D + g + q);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xFFFFFFFFu, lw, o);
+                    if (lane == 0) cs.l[q] += lw;
+                }
+            }
+            if (pass == 1) {
+                __syncthreads();
+                const int nj = ncc - base < 32 ? ncc - base : 32;
+#pragma unroll
+                for (int k = 0; k < kMaxOut; ++k) {
+                    const int idx = tid + k * kThreads;
+                    if (idx >= g * D) break;
+                    const int q = idx / D, d = idx - q * D;
+                    float a = acc[k];
+#pragma unroll 4
+                    for (int j = 0; j < nj; ++j) {
+                        const int s2 = cs.slot[j];
+                        if (s2 < 0) continue;
+                        a += cs.w[q][j] * __ldcg(p.partials + (int64_t)s2 * slot_floats + q * D + d);
+                    }
+                    acc[k] = a;
+                }
+            }
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int k = 0; k < kMaxOut; ++k) {
+        const int idx = tid + k * kThreads;
+        if (idx >= g * D) break;
+        const int q = idx / D, d = idx - q * D;
+        const float l = cs.l[q];
+        p.out[((int64_t)u.b * p.Hq + (int64_t)u.h * g + q) * D + d] = (l > 0.0f) ? acc[k] / l : 0.0f;
     }
 }
 
@@ -284,28 +476,14 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_attention_kern
     const int tig = lane & 3;
     const int B = p.B;
 
-    // ---- prologue: lookup tables, barriers, sequence lengths ----------------
+    // ---- prologue 1: barriers, sequence lengths, this CTA's tile range -----
     const float st_k = *p.st_k;
     const float st_v = *p.st_v;
-    {
-        uint8_t* lk = reinterpret_cast<uint8_t*>(sm.lut_k);
-        uint8_t* lv = reinterpret_cast<uint8_t*>(sm.lut_v);
-        for (int e = tid; e < 1024; e += kWarps * 32) {
-            lk[e] = (uint8_t)lut_entry((uint32_t)(e >> 3), (uint32_t)(e & 7), st_k);
-            lv[e] = (uint8_t)lut_entry((uint32_t)(e >> 3), (uint32_t)(e & 7), st_v);
-        }
-    }
-    if (tid == 0 && blockIdx.x == 0) {
-        const bool ok = st_k > 0.f && st_k <= 3.4028234663852886e38f && st_v > 0.f &&
-                        st_v <= 3.4028234663852886e38f;
-        if (!ok) report(p.status, NVFP4_ERR_NONFINITE);
-    }
     if (lane == 0) {
 #pragma unroll
         for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[warp][s], 1);
         fence_mbar_init();
     }
-    // lengths and the per-sequence tile prefix (units of one sequence are contiguous)
     {
         constexpr int per = (kMaxBatchPerLaunch + kWarps * 32 - 1) / (kWarps * 32);
         int tiles[per];
@@ -325,7 +503,6 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_attention_kern
             tiles[i] = (b < B) ? p.Hkv * (L > 0 ? (L + kTile - 1) / kTile : 1) : 0;
             run += tiles[i];
         }
-        // exclusive scan of `run` over the CTA
         int incl = run;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -354,20 +531,32 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_attention_kern
     const int64_t t_end = range_start(c + 1, T, N);
     if (t_begin >= t_end) return;
 
-    // ---- producer: lane 0 of each warp fills the warp's ring ---------------
+    // ---- prologue 2: lane 0 of each warp starts filling the warp's ring ----
     Cursor prod;
     prod.seg_lo = t_begin;
     prod.t_end = t_end;
     prod.done = false;
-    cursor_enter(prod, sm.prefix, sm.lens, B, p.Hkv, warp);
     uint32_t issued = 0;
     if (lane == 0) {
+        cursor_enter(prod, sm.prefix, sm.lens, B, p.Hkv, warp);
         for (int s = 0; s < kStages && !prod.done; ++s) {
             issue_tile<D>(p, prod.u, prod.gt, sm.ring[warp][s], &sm.bar[warp][s]);
             ++issued;
             cursor_next(prod, sm.prefix, sm.lens, B, p.Hkv, warp);
         }
     }
+
+    // ---- prologue 3: FP8 lookup tables, built while the first copies fly ---
+    for (int sb = tid; sb < 128; sb += kWarps * 32) {
+        sm.lut_k[sb] = lut_words((uint32_t)sb, st_k);
+        sm.lut_v[sb] = lut_words((uint32_t)sb, st_v);
+    }
+    if (tid == 0 && blockIdx.x == 0) {
+        const bool ok = st_k > 0.f && st_k <= 3.4028234663852886e38f && st_v > 0.f &&
+                        st_v <= 3.4028234663852886e38f;
+        if (!ok) report(p.status, NVFP4_ERR_NONFINITE);
+    }
+    __syncthreads();
 
     uint32_t consumed = 0;
     bool aborted = false;
@@ -378,9 +567,8 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_attention_kern
         const Unit u = find_unit(sm.prefix, sm.lens, B, p.Hkv, seg_lo);
         const int64_t seg_hi = u.U1 < t_end ? u.U1 : t_end;
 
-        uint32_t qf[KS][NT][2], ql[KS][NT][2];
-        float cscale[NT][2];
-        load_q<D, NT, QF32>(p, u.b, u.h, gid, tig, qf, ql, cscale);
+        QueryFrags<D, NT, QF32> qf;
+        load_q<D, NT, QF32>(p, u.b, u.h, gid, tig, qf);
 
         float o[KS][NT][4];
         float m_run[NT][2], l_run[NT][2];
@@ -417,137 +605,135 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_attention_kern
             const uint8_t* vc_s = st + G::OFF_VC;
             const uint8_t* ks_s = st + G::OFF_KS;
             const uint8_t* vs_s = st + G::OFF_VS;
+            const bool sub1 = valid > 16;
 
+            if (!aborted && valid > 0) {
+                // ---------------- S^T = K Q^T for both 16-token sub-tiles -----------
+                float sc[2][NT][4];
 #pragma unroll
-            for (int sub = 0; sub < kTile / 16; ++sub) {
-                if (aborted || sub * 16 >= valid) break;
-                // ---------------- K: dequantize this lane's A fragments -------------
-                const int r0 = sub * 16 + gid;
-                uint32_t fk[2][2 * G::WK];  // [token r0 / r0+8][fp8x4 words]
+                for (int sub = 0; sub < 2; ++sub) {
+                    if (sub == 1 && !sub1) break;
+                    uint32_t fk[2][D / 8];
+                    dequant_k<D>(kc_s, ks_s, sm.lut_k, sub, gid, tig, fk);
+                    float sh[NT][4], sl[NT][4];
 #pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    const int r = r0 + 8 * rr;
-                    uint32_t w[G::WK];
-                    if constexpr (D == 128) {
-                        const uint4 x = *reinterpret_cast<const uint4*>(kc_s + r * G::KB + 16 * tig);
-                        w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) sh[nt][k] = sl[nt][k] = 0.0f;
+                    if constexpr (QF32) {
+#pragma unroll
+                        for (int s = 0; s < KS; ++s) {
+                            uint32_t a0, a2, a1, a3;
+                            e4m3x4_to_f16x2x2(fk[0][s], a0, a2);
+                            e4m3x4_to_f16x2x2(fk[1][s], a1, a3);
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) {
+                                mma_f16_16816(sh[nt], a0, a1, a2, a3, qf.hi[s][nt][0], qf.hi[s][nt][1]);
+                                mma_f16_16816(sl[nt], a0, a1, a2, a3, qf.lo[s][nt][0], qf.lo[s][nt][1]);
+                            }
+                        }
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) sc[sub][nt][k] = sh[nt][k] + sl[nt][k];
                     } else {
-                        const uint2 x = *reinterpret_cast<const uint2*>(kc_s + r * G::KB + 8 * tig);
-                        w[0] = x.x; w[1] = x.y;
-                    }
 #pragma unroll
-                    for (int j = 0; j < G::WK; ++j) {
-                        const int blk = (G::EK * tig + 8 * j) / 16;
-                        const uint2 lut = sm.lut_k[ks_s[r * G::SB + blk] & 0x7F];
-                        dequant_word(w[j], lut.x, lut.y, fk[rr][2 * j], fk[rr][2 * j + 1]);
-                    }
-                }
-                // ---------------- S^T = K Q^T on tensor cores -----------------------
-                float sacc[NT][4];
+                        for (int s = 0; s < D / 32; ++s) {
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+                            for (int nt = 0; nt < NT; ++nt) {
+                                mma_e4m3_16832(sh[nt], fk[0][2 * s], fk[1][2 * s], fk[0][2 * s + 1],
+                                               fk[1][2 * s + 1], qf.hi[s][nt][0], qf.hi[s][nt][1]);
+                                mma_e4m3_16832(sl[nt], fk[0][2 * s], fk[1][2 * s], fk[0][2 * s + 1],
+                                               fk[1][2 * s + 1], qf.lo[s][nt][0], qf.lo[s][nt][1]);
+                            }
+                        }
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) sacc[nt][k] = 0.0f;
+                        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int s = 0; s < KS; ++s) {
-                    const uint32_t a0 = lo16_to_f16x2(fk[0][s]);
-                    const uint32_t a2 = hi16_to_f16x2(fk[0][s]);
-                    const uint32_t a1 = lo16_to_f16x2(fk[1][s]);
-                    const uint32_t a3 = hi16_to_f16x2(fk[1][s]);
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        mma_f16_16816(sacc[nt], a0, a1, a2, a3, qf[s][nt][0], qf[s][nt][1]);
-                        if (QF32) mma_f16_16816(sacc[nt], a0, a1, a2, a3, ql[s][nt][0], ql[s][nt][1]);
+                            for (int k = 0; k < 4; ++k) sc[sub][nt][k] = fmaf(sl[nt][k], 0.0625f, sh[nt][k]);
                     }
                 }
-                // ---------------- online softmax (base 2, lazy max) -----------------
-                const bool row0_ok = (sub * 16 + gid) < valid;
-                const bool row1_ok = (sub * 16 + gid + 8) < valid;
+                // ---------------- online softmax over the 32 tokens (base 2) -------
                 bool need = false;
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    sacc[nt][0] = row0_ok ? sacc[nt][0] * cscale[nt][0] : -INFINITY;
-                    sacc[nt][1] = row0_ok ? sacc[nt][1] * cscale[nt][1] : -INFINITY;
-                    sacc[nt][2] = row1_ok ? sacc[nt][2] * cscale[nt][0] : -INFINITY;
-                    sacc[nt][3] = row1_ok ? sacc[nt][3] * cscale[nt][1] : -INFINITY;
-                    need |= fmaxf(sacc[nt][0], sacc[nt][2]) > m_run[nt][0] + kRescaleSlack;
-                    need |= fmaxf(sacc[nt][1], sacc[nt][3]) > m_run[nt][1] + kRescaleSlack;
+                for (int sub = 0; sub < 2; ++sub) {
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int row = sub * 16 + gid + 8 * (k >> 1);
+                            const float v = (sub == 0 || sub1) ? sc[sub][nt][k] : 0.0f;
+                            sc[sub][nt][k] = row < valid ? v * qf.cscale[nt][k & 1] : -INFINITY;
+                            need |= sc[sub][nt][k] > m_run[nt][k & 1] + kRescaleSlack;
+                        }
+                    }
                 }
                 if (__any_sync(0xFFFFFFFFu, need)) {
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-                        for (int k = 0; k < 2; ++k) {
-                            float mx = fmaxf(sacc[nt][k], sacc[nt][k + 2]);
+                        for (int col = 0; col < 2; ++col) {
+                            float mx = fmaxf(fmaxf(sc[0][nt][col], sc[0][nt][col + 2]),
+                                             fmaxf(sc[1][nt][col], sc[1][nt][col + 2]));
                             mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 4));
                             mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 8));
                             mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
-                            const float m_new = fmaxf(m_run[nt][k], mx);
-                            const float f = (m_run[nt][k] == -INFINITY) ? 0.0f : fast_exp2(m_run[nt][k] - m_new);
-                            m_run[nt][k] = m_new;
-                            l_run[nt][k] *= f;
+                            const float m_new = fmaxf(m_run[nt][col], mx);
+                            const float f = (m_run[nt][col] == -INFINITY) ? 0.0f : fast_exp2(m_run[nt][col] - m_new);
+                            m_run[nt][col] = m_new;
+                            l_run[nt][col] *= f;
 #pragma unroll
                             for (int i = 0; i < KS; ++i) {
-                                o[i][nt][k] *= f;
-                                o[i][nt][k + 2] *= f;
+                                o[i][nt][col] *= f;
+                                o[i][nt][col + 2] *= f;
                             }
                         }
                     }
                 }
-                uint32_t bph[NT][2], bpl[NT][2];
+                // ---------------- P (hi + lo f16) and O^T += V^T P^T ---------------
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    float pv[4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        pv[k] = fast_exp2(sacc[nt][k] - m_run[nt][k & 1]);
-                        l_run[nt][k & 1] += pv[k];
-                    }
-                    const uint32_t h01 = pack_f16x2(pv[0], pv[1]);
-                    const uint32_t h23 = pack_f16x2(pv[2], pv[3]);
-                    const uint32_t l01 = pack_f16x2(pv[0] - f16_lo_to_float(h01), pv[1] - f16_hi_to_float(h01));
-                    const uint32_t l23 = pack_f16x2(pv[2] - f16_lo_to_float(h23), pv[3] - f16_hi_to_float(h23));
-                    bph[nt][0] = movmatrix_trans(h01);
-                    bph[nt][1] = movmatrix_trans(h23);
-                    bpl[nt][0] = movmatrix_trans(l01);
-                    bpl[nt][1] = movmatrix_trans(l23);
-                }
-                // ---------------- V: dequantize token pairs for the A fragments -----
-                // lane (gid, tig) covers tokens 2tig, 2tig+1, 2tig+8, 2tig+9 of the
-                // sub-tile and channels [EV*gid, EV*gid + EV) (one scale block)
-                uint32_t gv[4][2 * G::WV];
-#pragma unroll
-                for (int tt = 0; tt < 4; ++tt) {
-                    const int r = sub * 16 + 2 * tig + (tt & 1) + 8 * (tt >> 1);
-                    const uint2 lut = sm.lut_v[vs_s[r * G::SB + (G::EV * gid) / 16] & 0x7F];
-                    if constexpr (D == 128) {
-                        const uint2 x = *reinterpret_cast<const uint2*>(vc_s + r * G::KB + 8 * gid);
-                        dequant_word(x.x, lut.x, lut.y, gv[tt][0], gv[tt][1]);
-                        dequant_word(x.y, lut.x, lut.y, gv[tt][2], gv[tt][3]);
-                    } else {
-                        const uint32_t x = *reinterpret_cast<const uint32_t*>(vc_s + r * G::KB + 4 * gid);
-                        dequant_word(x, lut.x, lut.y, gv[tt][0], gv[tt][1]);
-                    }
-                }
-                // ---------------- O^T += V^T P^T on tensor cores --------------------
-#pragma unroll
-                for (int i = 0; i < KS; ++i) {
-                    // row gid <-> channel i, row gid + 8 <-> channel KS + i (of the lane's EV)
-                    const int e0 = i, e1 = KS + i;
-                    const uint32_t sel0 = (e0 & 2) ? 0x7362u : 0x5140u;
-                    const uint32_t sel1 = (e1 & 2) ? 0x7362u : 0x5140u;
-                    const uint32_t p00 = __byte_perm(gv[0][e0 >> 2], gv[1][e0 >> 2], sel0);
-                    const uint32_t p01 = __byte_perm(gv[0][e1 >> 2], gv[1][e1 >> 2], sel1);
-                    const uint32_t p10 = __byte_perm(gv[2][e0 >> 2], gv[3][e0 >> 2], sel0);
-                    const uint32_t p11 = __byte_perm(gv[2][e1 >> 2], gv[3][e1 >> 2], sel1);
-                    const uint32_t a0 = (e0 & 1) ? hi16_to_f16x2(p00) : lo16_to_f16x2(p00);
-                    const uint32_t a1 = (e1 & 1) ? hi16_to_f16x2(p01) : lo16_to_f16x2(p01);
-                    const uint32_t a2 = (e0 & 1) ? hi16_to_f16x2(p10) : lo16_to_f16x2(p10);
-                    const uint32_t a3 = (e1 & 1) ? hi16_to_f16x2(p11) : lo16_to_f16x2(p11);
+                for (int sub = 0; sub < 2; ++sub) {
+                    if (sub == 1 && !sub1) break;
+                    uint32_t bph[NT][2], bpl[NT][2];
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        mma_f16_16816(o[i][nt], a0, a1, a2, a3, bph[nt][0], bph[nt][1]);
-                        mma_f16_16816(o[i][nt], a0, a1, a2, a3, bpl[nt][0], bpl[nt][1]);
+                        float pv[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            pv[k] = fast_exp2(sc[sub][nt][k] - m_run[nt][k & 1]);
+                            l_run[nt][k & 1] += pv[k];
+                        }
+                        const uint32_t h01 = pack_f16x2(pv[0], pv[1]);
+                        const uint32_t h23 = pack_f16x2(pv[2], pv[3]);
+                        const uint32_t l01 = pack_f16x2(pv[0] - f16_lo_to_float(h01), pv[1] - f16_hi_to_float(h01));
+                        const uint32_t l23 = pack_f16x2(pv[2] - f16_lo_to_float(h23), pv[3] - f16_hi_to_float(h23));
+                        bph[nt][0] = movmatrix_trans(h01);
+                        bph[nt][1] = movmatrix_trans(h23);
+                        bpl[nt][0] = movmatrix_trans(l01);
+                        bpl[nt][1] = movmatrix_trans(l23);
+                    }
+                    uint32_t gv[4][D / 32];
+                    dequant_v<D>(vc_s, vs_s, sm.lut_v, sub, gid, tig, gv);
+                    // m-tile i: row gid <-> channel i, row gid + 8 <-> channel KS + i
+                    // (of the lane's EV channels); consecutive tokens pair up in f16x2
+#pragma unroll
+                    for (int i = 0; i < KS; i += 2) {
+                        const int e0 = i, e1 = KS + i;
+                        const uint32_t sel0 = (e0 & 2) ? 0x7362u : 0x5140u;
+                        const uint32_t sel1 = (e1 & 2) ? 0x7362u : 0x5140u;
+                        uint32_t a0[2], a1[2], a2[2], a3[2];
+                        e4m3x4_to_f16x2x2(__byte_perm(gv[0][e0 >> 2], gv[1][e0 >> 2], sel0), a0[0], a0[1]);
+                        e4m3x4_to_f16x2x2(__byte_perm(gv[0][e1 >> 2], gv[1][e1 >> 2], sel1), a1[0], a1[1]);
+                        e4m3x4_to_f16x2x2(__byte_perm(gv[2][e0 >> 2], gv[3][e0 >> 2], sel0), a2[0], a2[1]);
+                        e4m3x4_to_f16x2x2(__byte_perm(gv[2][e1 >> 2], gv[3][e1 >> 2], sel1), a3[0], a3[1]);
+#pragma unroll
+                        for (int ii = 0; ii < 2; ++ii) {
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) {
+                                mma_f16_16816(o[i + ii][nt], a0[ii], a1[ii], a2[ii], a3[ii], bph[nt][0], bph[nt][1]);
+                                mma_f16_16816(o[i + ii][nt], a0[ii], a1[ii], a2[ii], a3[ii], bpl[nt][0], bpl[nt][1]);
+                            }
+                        }
                     }
                 }
             }
@@ -603,8 +789,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_attention_kern
 #pragma unroll
                 for (int w = 0; w < kWarps; ++w) {
                     const float mw = sm.merge_m[w][q];
-                    if (mw == -INFINITY) continue;
-                    const float f = fast_exp2(mw - M);
+                    const float f = (mw == -INFINITY) ? 0.0f : fast_exp2(mw - M);
                     acc += f * sm.merge_o[w][q][d];
                     l += f * sm.merge_l[w][q];
                 }
@@ -623,11 +808,11 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_attention_kern
         if (!whole) {
             __threadfence();
             __syncthreads();
+            const int64_t c_first = cta_of(u.U0, T, N);
+            const int64_t c_last = cta_of(u.U1 - 1, T, N);
             if (tid == 0) {
                 // contributors: the CTAs with a non-empty range inside the unit's
                 // span (ranges are empty only when there are fewer tiles than CTAs)
-                const int64_t c_first = cta_of(u.U0, T, N);
-                const int64_t c_last = cta_of(u.U1 - 1, T, N);
                 int contributors = 0;
                 for (int64_t cc = c_first; cc <= c_last; ++cc)
                     contributors += range_start(cc, T, N) < range_start(cc + 1, T, N);
@@ -637,31 +822,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_attention_kern
             __syncthreads();
             if (sm.last_flag) {
                 __threadfence();
-                const int64_t c_first = cta_of(u.U0, T, N);
-                const int64_t c_last = cta_of(u.U1 - 1, T, N);
-                for (int idx = tid; idx < g * D; idx += kWarps * 32) {
-                    const int q = idx / D, d = idx - q * D;
-                    float M = -INFINITY;
-                    for (int64_t cc = c_first; cc <= c_last; ++cc) {
-                        if (range_start(cc, T, N) == range_start(cc + 1, T, N)) continue;
-                        const int64_t sl = partial_slot(cc, u.U0, T, N);
-                        M = fmaxf(M, __ldcg(p.partials + sl * slot_floats + g * D + q));
-                    }
-                    float acc = 0.0f, l = 0.0f;
-                    if (M != -INFINITY) {
-                        for (int64_t cc = c_first; cc <= c_last; ++cc) {
-                            if (range_start(cc, T, N) == range_start(cc + 1, T, N)) continue;
-                            const int64_t sl = partial_slot(cc, u.U0, T, N);
-                            const float* part = p.partials + sl * slot_floats;
-                            const float mw = __ldcg(part + g * D + q);
-                            if (mw == -INFINITY) continue;
-                            const float f = fast_exp2(mw - M);
-                            acc += f * __ldcg(part + q * D + d);
-                            l += f * __ldcg(part + g * D + g + q);
-                        }
-                    }
-                    p.out[((int64_t)u.b * p.Hq + (int64_t)u.h * g + q) * D + d] = (l > 0.0f) ? acc / l : 0.0f;
-                }
+                combine_partials<D, NT>(p, sm.comb, u, T, N, c_first, c_last, slot_floats, tid, warp, lane);
                 if (tid == 0) atomicExch(&p.counters[(int64_t)u.b * p.Hkv + u.h], 0);
             }
         }

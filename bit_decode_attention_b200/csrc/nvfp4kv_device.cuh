@@ -82,13 +82,24 @@ __device__ __forceinline__ uint32_t e2m1_from_float(float y) {
 // NVFP4 -> FP8 lookup
 // ---------------------------------------------------------------------------
 // The FP8 value of a code depends only on its 3-bit magnitude, the block's
-// scale byte and the tensor scale.  lut_entry(sb, m, st) is that value for one
-// magnitude; a block's 8 entries fit two 32-bit words, which `byte_perm` then
-// indexes with four 3-bit selectors at a time.
-__device__ __forceinline__ uint32_t lut_entry(uint32_t sb, uint32_t m3, float s_tensor) {
-    if ((sb & 0x7Fu) == 0x7Fu) return 0u;                    // never written by quantize
-    const float prod = __fmul_rn(e2m1_magnitude(m3), e4m3_to_float(sb & 0x7Fu)); // exact
-    return e4m3_from_float(__fmul_rn(prod, s_tensor));
+// scale byte and the tensor scale:  E4M3(fl32(fl32(|c| * value(sb)) * s)).
+// A block's 8 values fit two 32-bit words (byte m = magnitude m), which
+// `byte_perm` then indexes with four 3-bit selectors at a time.
+// |c| * value(sb) has at most 6 significant bits, so the first product is
+// exact; the second is one fp32 rounding; the E4M3 conversion rounds to
+// nearest even and saturates at 448.
+__device__ __forceinline__ uint2 lut_words(uint32_t sb, float s_tensor) {
+    if ((sb & 0x7Fu) == 0x7Fu) return make_uint2(0u, 0u);   // never written by quantize
+    const float v = e4m3_to_float(sb & 0x7Fu);
+    float f[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) f[m] = __fmul_rn(__fmul_rn(e2m1_magnitude((uint32_t)m), v), s_tensor);
+    uint16_t b01, b23, b45, b67;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(b01) : "f"(f[1]), "f"(f[0]));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(b23) : "f"(f[3]), "f"(f[2]));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(b45) : "f"(f[5]), "f"(f[4]));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(b67) : "f"(f[7]), "f"(f[6]));
+    return make_uint2((uint32_t)b01 | ((uint32_t)b23 << 16), (uint32_t)b45 | ((uint32_t)b67 << 16));
 }
 
 // Dequantize 8 packed codes (one 32-bit word; element k in nibble k) to 8 FP8
@@ -168,18 +179,21 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Two E4M3 bytes (lo, hi of a 16-bit value) -> f16x2 (exact).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
-    uint32_t r;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
-    return r;
+// Four E4M3 bytes -> two f16x2 (exact): lo = bytes (0, 1), hi = bytes (2, 3),
+// the lower-addressed byte in the low half.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(x));
 }
 
-__device__ __forceinline__ uint32_t lo16_to_f16x2(uint32_t x) {
-    return e4m3x2_to_f16x2(static_cast<uint16_t>(x & 0xFFFFu));
-}
-__device__ __forceinline__ uint32_t hi16_to_f16x2(uint32_t x) {
-    return e4m3x2_to_f16x2(static_cast<uint16_t>(x >> 16));
+// Two floats -> two E4M3 bytes (lo in the low byte), round to nearest even,
+// finite overflow saturates.  Used for query operands only.
+__device__ __forceinline__ uint32_t e4m3x2_from_floats(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
 }
 
 // Two floats -> f16x2 (lo in the low half), round to nearest even.
@@ -204,15 +218,23 @@ __device__ __forceinline__ float f16_hi_to_float(uint32_t x) {
 // lane/4, columns 2*(lane%4), +1).
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
     uint32_t r;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
     return r;
 }
 
 // D += A(16x16, f16, row) * B(16x8, f16, col), fp32 accumulate.
 __device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                               uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D += A(16x32, e4m3, row) * B(32x8, e4m3, col), fp32 accumulate.
+__device__ __forceinline__ void mma_e4m3_16832(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 "
         "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));

@@ -220,9 +220,7 @@ __global__ void __launch_bounds__(256) dequant_fp8_kernel(
     uint8_t* __restrict__ out, int32_t* __restrict__ status) {
     __shared__ uint2 lut[128];
     const float st = *s_tensor_p;
-    uint8_t* lut_bytes = reinterpret_cast<uint8_t*>(lut);
-    for (int e = threadIdx.x; e < 1024; e += blockDim.x)
-        lut_bytes[e] = (uint8_t)lut_entry((uint32_t)(e >> 3), (uint32_t)(e & 7), st);
+    for (int sb = threadIdx.x; sb < 128; sb += blockDim.x) lut[sb] = lut_words((uint32_t)sb, st);
     if (blockIdx.x == 0 && threadIdx.x == 0 && !(st > 0.0f && st <= 3.4028234663852886e38f))
         report(status, NVFP4_ERR_NONFINITE);
     __syncthreads();
