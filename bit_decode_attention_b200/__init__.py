@@ -25,7 +25,7 @@ from ._native import (NVFP4_ERR_CAPACITY, NVFP4_ERR_INVALID_ARG, NVFP4_ERR_NONFI
 __all__ = [
     "KVPlane", "nvfp4_cache_bytes", "nvfp4_calib_tensor_scale", "nvfp4_kv_quantize_append",
     "nvfp4_kv_dequant_fp8", "nvfp4_decode_attention_workspace", "nvfp4_decode_attention",
-    "nvfp4_version", "NativeError",
+    "nvfp4_version", "NativeError", "nvfp4_decode_attention_noalloc",
 ]
 
 
@@ -157,4 +157,24 @@ def nvfp4_decode_attention(q: torch.Tensor, k: KVPlane, v: KVPlane, s_tensor_k: 
         _ptr(s_tensor_v), _ptr(seq_lens), ctypes.c_float(softmax_scale), _ptr(out),
         _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
     _native.check("nvfp4_decode_attention", st)
+    return out
+
+
+def nvfp4_decode_attention_noalloc(q: torch.Tensor, k: KVPlane, v: KVPlane, s_tensor_k: torch.Tensor,
+                                   s_tensor_v: torch.Tensor, seq_lens: torch.Tensor,
+                                   softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                                   status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """nvfp4_decode_attention without a workspace, for callers that may not
+    allocate device memory: scratch is the library's built-in device buffer
+    (shared by all calls on a device; calls must not overlap on the GPU)."""
+    _need_cuda(q, s_tensor_k, s_tensor_v, seq_lens, out, status)
+    B, H_q, D = q.shape
+    if out is None:
+        out = torch.empty(B, H_q, D, dtype=torch.float32, device=q.device)
+    kp, vp = k.struct(), v.struct()
+    st = _native.lib().nvfp4_decode_attention_noalloc(
+        _ptr(q), _dtype_code(q), H_q, ctypes.byref(kp), ctypes.byref(vp), _ptr(s_tensor_k),
+        _ptr(s_tensor_v), _ptr(seq_lens), ctypes.c_float(softmax_scale), _ptr(out), _ptr(status),
+        _stream(stream))
+    _native.check("nvfp4_decode_attention_noalloc", st)
     return out

@@ -32,6 +32,7 @@ EXPORTS = (
     "nvfp4_kv_dequant_fp8",
     "nvfp4_decode_attention_workspace",
     "nvfp4_decode_attention",
+    "nvfp4_decode_attention_noalloc",
 )
 
 
@@ -84,6 +85,9 @@ def lib():
     L.nvfp4_decode_attention.argtypes = [vp, i32, i32, plane_p, plane_p, vp, vp, vp, f32, vp, vp,
                                          sz, vp, vp]
     L.nvfp4_decode_attention.restype = i32
+    L.nvfp4_decode_attention_noalloc.argtypes = [vp, i32, i32, plane_p, plane_p, vp, vp, vp, f32, vp,
+                                                 vp, vp]
+    L.nvfp4_decode_attention_noalloc.restype = i32
     _lib = L
     return L
 

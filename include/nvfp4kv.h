@@ -175,6 +175,35 @@ nvfp4_status nvfp4_decode_attention(const void* q, nvfp4_dtype q_dtype, int H_q,
                                     float* out, void* workspace, size_t workspace_bytes,
                                     int32_t* d_status, nvfp4_stream_t stream);
 
+/* Decode attention for callers that cannot allocate device memory.
+ *
+ * The pages describe no such call; it exists for users of this library whose
+ * code may not call cudaMalloc or any allocating routine -- code running inside
+ * a framework or host whose memory pool owns every device allocation, plugins
+ * that receive only their input and output buffers, or paths that must not
+ * allocate while other work is in flight.
+ *
+ * Same arguments and results as nvfp4_decode_attention, without the workspace:
+ * the split-K partial results and arrival counters live in one file-scope
+ * device array of NVFP4_NOALLOC_SCRATCH_BYTES (8 MiB), held by every GPU that
+ * loads this library until the process exits.  Behaviour:
+ *   - Shapes whose workspace (nvfp4_decode_attention_workspace) exceeds the
+ *     buffer are rejected with NVFP4_ERR_WORKSPACE before anything is queued.
+ *   - The first call on each device looks up the buffer's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - Each call clears the arrival counters with a memset on `stream`, then
+ *     runs the same kernel as nvfp4_decode_attention.
+ *   - Every call on a device shares the one buffer and leaves its contents
+ *     behind: calls whose execution overlaps on the GPU (other streams, other
+ *     host threads) race and give wrong results; serialize them.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+#define NVFP4_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+nvfp4_status nvfp4_decode_attention_noalloc(const void* q, nvfp4_dtype q_dtype, int H_q,
+                                            const nvfp4_kv_plane* k, const nvfp4_kv_plane* v,
+                                            const float* d_s_tensor_k, const float* d_s_tensor_v,
+                                            const int32_t* d_seq_lens, float softmax_scale,
+                                            float* out, int32_t* d_status, nvfp4_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
