@@ -30,7 +30,7 @@ int device_sm_count() {
 AttnWorkspace attention_workspace(int B, int Hq, int Hkv, int D) {
     AttnWorkspace w{};
     const int g = Hq / Hkv;
-    w.grid = kCtasPerSm * device_sm_count();
+    w.grid = kMaxCtasPerSm * device_sm_count();
     w.counters_bytes = ((size_t)B * Hkv * sizeof(int32_t) + 255) / 256 * 256;
     w.partial_floats = (size_t)2 * w.grid * g * (D + 2);
     w.total_bytes = w.counters_bytes + w.partial_floats * sizeof(float);

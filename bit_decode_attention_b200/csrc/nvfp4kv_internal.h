@@ -13,8 +13,11 @@ namespace nvfp4kv {
 constexpr int kTile = 32;
 // sequences handled by one decode-attention launch
 constexpr int kMaxBatchPerLaunch = 512;
-// resident decode-attention CTAs per SM (the kernel is written for this)
+// resident decode-attention CTAs per SM (the warp-MMA kernel is written for
+// this); workspace partial slots are sized for the largest grid any of the
+// decode-attention kernels launches (kMaxCtasPerSm x SM count)
 constexpr int kCtasPerSm = 2;
+constexpr int kMaxCtasPerSm = 3;
 
 int device_sm_count();  // multiprocessor count of the current device (cached)
 

@@ -221,3 +221,18 @@ def test_attention_length_past_capacity_reports(nv):
     torch.cuda.synchronize()
     assert status.item() == nv.NVFP4_ERR_CAPACITY
     assert torch.isfinite(out).all().item()
+
+
+@pytest.mark.parametrize("D,q_dtype", [(128, "bf16"), (128, "f32"), (64, "bf16")])
+def test_attention_ignores_bytes_past_the_sequence(nv, D, q_dtype):
+    # cache slots past each sequence's length hold 0xFF bytes (E4M3 NaN scales,
+    # code -6): the output must not see them, P = 0 there must not meet a NaN V
+    c = Case(synthetic.shrink(synthetic.get("gqa"), B=3, Hq=16, Hkv=2, D=D), lens=[130, 1, 259],
+             q_dtype=q_dtype)
+    for b, L in enumerate(c.lens):
+        for plane in (c.k, c.v):
+            plane.codes[b, :, L:] = 0xFF
+            plane.scales[b, :, L:] = 0xFF
+    got = c.gpu_attention().cpu().numpy()
+    assert c.status.item() == 0
+    assert_attention_close(got, c.oracle_attention())
