@@ -32,7 +32,7 @@ AttnWorkspace attention_workspace(int B, int Hq, int Hkv, int D) {
     const int g = Hq / Hkv;
     w.grid = kMaxCtasPerSm * device_sm_count();
     w.counters_bytes = ((size_t)B * Hkv * sizeof(int32_t) + 255) / 256 * 256;
-    w.partial_floats = (size_t)2 * w.grid * g * (D + 2);
+    w.partial_floats = (size_t)2 * w.grid * (size_t)partial_slot_floats(g, D);
     w.total_bytes = w.counters_bytes + w.partial_floats * sizeof(float);
     return w;
 }
@@ -139,7 +139,7 @@ nvfp4_status nvfp4_decode_attention(const void* q, nvfp4_dtype q_dtype, int H_q,
     if (!(std::isfinite(softmax_scale)) || softmax_scale < 0.0f) return NVFP4_ERR_INVALID_ARG;
     const int B = k->B;
     if (B == 0) return NVFP4_OK;
-    if (q == nullptr || out == nullptr || !aligned16(q)) return NVFP4_ERR_INVALID_ARG;
+    if (q == nullptr || out == nullptr || !aligned16(q) || !aligned16(out)) return NVFP4_ERR_INVALID_ARG;
     const AttnWorkspace ws = attention_workspace(B, H_q, k->H_kv, k->D);
     if (workspace == nullptr || workspace_bytes < ws.total_bytes || !aligned16(workspace))
         return NVFP4_ERR_WORKSPACE;

@@ -110,11 +110,11 @@ __device__ __forceinline__ uint2 lut_words(uint32_t sb, float s_tensor) {
 //     byte permutes of (x << 4, x) move bits 3/7/11/15 (19/23/27/31) there.
 __device__ __forceinline__ void dequant_word(uint32_t x, uint32_t lut_lo, uint32_t lut_hi,
                                              uint32_t& out_lo, uint32_t& out_hi) {
-    const uint32_t sel_lo = x & 0x7777u;
-    const uint32_t sel_hi = (x >> 16) & 0x7777u;
+    const uint32_t sel_lo = x & 0x77777777u;
+    const uint32_t sel_hi = __umulhi(sel_lo, 0x10000u);   // >> 16 on the multiply pipe
     const uint32_t mag_lo = __byte_perm(lut_lo, lut_hi, sel_lo);
     const uint32_t mag_hi = __byte_perm(lut_lo, lut_hi, sel_hi);
-    const uint32_t xs = x << 4;
+    const uint32_t xs = x * 16u;
     const uint32_t sgn_lo = __byte_perm(xs, x, 0x5140u);
     const uint32_t sgn_hi = __byte_perm(xs, x, 0x7362u);
     out_lo = mag_lo | (sgn_lo & 0x80808080u);

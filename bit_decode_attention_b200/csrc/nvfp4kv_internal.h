@@ -21,6 +21,12 @@ constexpr int kMaxCtasPerSm = 3;
 
 int device_sm_count();  // multiprocessor count of the current device (cached)
 
+// floats per split-K partial slot: O [g][D], m [g], l [g], padded to a whole
+// float4 so that every slot starts 16-byte aligned
+__host__ __device__ constexpr int64_t partial_slot_floats(int g, int D) {
+    return ((int64_t)g * (D + 2) + 3) / 4 * 4;
+}
+
 cudaError_t launch_calib(const void* x, bool f32, int64_t n, float* d_s_tensor, int32_t* d_status,
                          cudaStream_t stream);
 
@@ -42,7 +48,7 @@ struct AttnLaunch {
     const int32_t* seq_lens;
     float softmax_scale;
     float* out;
-    float* partials;     // [2 * grid][g][D + 2]
+    float* partials;     // [2 * grid] slots of partial_slot_floats(g, D)
     int32_t* counters;   // [B * Hkv], zero between calls
     int32_t* status;
     int grid;            // CTAs
@@ -53,7 +59,7 @@ cudaError_t launch_decode_attention(const AttnLaunch& a, cudaStream_t stream);
 // workspace layout of nvfp4_decode_attention for one shape
 struct AttnWorkspace {
     size_t counters_bytes;  // B * H_kv int32, padded to 256 bytes
-    size_t partial_floats;  // 2 * grid * g * (D + 2)
+    size_t partial_floats;  // 2 * grid * partial_slot_floats(g, D)
     size_t total_bytes;
     int grid;
 };

@@ -163,11 +163,11 @@ size_t nvfp4_decode_attention_workspace(int B, int H_q, int H_kv, int D);
  *   d_s_tensor_k, d_s_tensor_v  device floats
  *   d_seq_lens   device int32 [B], tokens to attend per sequence (<= S_max)
  *   softmax_scale  0 selects 1/sqrt(D)
- *   out          device float [B][H_q][D]
+ *   out          device float [B][H_q][D], 16-byte aligned
  *   workspace    device, >= nvfp4_decode_attention_workspace(...) bytes,
  *                zero-filled once (see above), 16-byte aligned
  * Lengths past S_max are clamped and reported as NVFP4_ERR_CAPACITY.
- * Batches larger than 1024 sequences are processed in launches of 1024. */
+ * Batches larger than 512 sequences are processed in launches of 512. */
 nvfp4_status nvfp4_decode_attention(const void* q, nvfp4_dtype q_dtype, int H_q,
                                     const nvfp4_kv_plane* k, const nvfp4_kv_plane* v,
                                     const float* d_s_tensor_k, const float* d_s_tensor_v,

@@ -94,6 +94,8 @@ def test_argument_validation_without_gpu(lib):
     assert at(*args(3, k, v, dev, 1 << 30)) == INVALID            # H_q % H_kv
     assert at(*args(4, k, v_other, dev, 1 << 30)) == INVALID      # planes disagree
     assert at(*args(2 * 17, k, v, dev, 1 << 30)) == _native.NVFP4_ERR_UNSUPPORTED
+    assert at(dev, 0, 4, ctypes.byref(k), ctypes.byref(v), dev, dev, dev, ctypes.c_float(0.0),
+              ctypes.c_void_p(68), dev, 1 << 30, None, None) == INVALID   # out misaligned
     assert at(*args(4, k, v, None, 0)) == WS
     assert at(*args(4, k, v, dev, 16)) == WS
     cal = lib.nvfp4_calib_tensor_scale
