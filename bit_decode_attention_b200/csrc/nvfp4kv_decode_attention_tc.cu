@@ -15,11 +15,11 @@
 // consecutive tiles overlap; they hand tiles to each other through
 // mbarriers (double-buffered operands), never through CTA-wide barriers:
 //
-//   load warp   : bulk copies of K/V codes and scale bytes into a 5-stage ring
+//   load warp   : bulk copies of K/V codes and scale bytes into a 4-stage ring
 //   dequant warps 0-3 and 8-11: thread t of group h = token t, head_dim half
 //                 h.  K codes -> signed FP8 K in tensor memory lane t (the A
 //                 operand of Q.K^T); V codes -> FP8 V^T in shared memory (the
-//                 MN-major A operand of P.V).  Operands are triple-buffered
+//                 MN-major A operand of P.V).  K and V^T have 5 buffers
 //   MMA warp    : S^T[t][n] = K . Q'^T,  O^T[d][n] += V^T . P^T
 //                 (a tcgen05 MMA costs about the same for any N up to 256:
 //                 the instruction count per tile, 4 + 4, sets the pace)
@@ -48,8 +48,10 @@ constexpr int STAGE = TILE * (2 * kKB + 2 * kSB);     // 18432
 constexpr int OFF_VC = TILE * kKB;
 constexpr int OFF_KS = 2 * TILE * kKB;
 constexpr int OFF_VS = 2 * TILE * kKB + TILE * kSB;
-constexpr int kStages = 5;
-constexpr int kBuf = 3;                               // K, S, V^T and P buffers
+constexpr int kStages = 4;
+// operand buffers: K (tensor memory) and V^T (shared memory) let the dequant
+// warps run ahead of the softmax; S (tensor memory) lets Q.K^T run ahead
+constexpr int kKBuf = 5, kVBuf = 5, kSBuf = 3, kPBuf = 3;
 constexpr int NTERM = 3;                              // E4M3 terms of P
 
 // warp roles
@@ -61,16 +63,17 @@ constexpr int kThreads = 14 * 32;
 constexpr int kSoftmaxBar = 1;                        // named barrier of the softmax warps
 
 constexpr uint32_t kWaitPolls = 1u << 16;             // sleeping polls (<= 20 us each) per wait
+constexpr uint32_t kMmaIdlePolls = 1u << 25;          // idle polls (~32 ns sleep each) of the MMA thread
 
 template <int NT>
 struct Cfg {
     static constexpr int NQ = 8 * NT;                 // query rows (padded GQA group)
     static constexpr int NS = 2 * NQ;                 // score columns: hi, lo
     static constexpr int NP = (NTERM * NQ + 15) / 16 * 16;   // P columns (MMA N), term-major
-    static constexpr uint32_t COL_K = 0;              // kBuf buffers x 32 columns (4 FP8 each)
-    static constexpr uint32_t COL_S = 32 * kBuf;      // kBuf buffers x NS
-    static constexpr uint32_t COL_O = COL_S + kBuf * NS;   // NP
-    static constexpr uint32_t kTmemCols = COL_O + NP <= 128 ? 128 : 256;
+    static constexpr uint32_t COL_K = 0;              // kKBuf buffers x 32 columns (4 FP8 each)
+    static constexpr uint32_t COL_S = 32 * kKBuf;     // kSBuf buffers x NS
+    static constexpr uint32_t COL_O = COL_S + kSBuf * NS;  // NP
+    static constexpr uint32_t kTmemCols = COL_O + NP <= 128 ? 128 : (COL_O + NP <= 256 ? 256 : 512);
     static_assert(COL_O + NP <= kTmemCols, "tensor memory columns");
 };
 
@@ -82,12 +85,13 @@ template <int NT>
 struct __align__(1024) Smem {
     using C = Cfg<NT>;
     uint8_t ring[kStages][STAGE];
-    uint8_t vt[kBuf][128 * TILE];                        // V^T: (d/16)*2048 + (t/8)*128 + (t%8)*16 + d%16
-    uint8_t pb[kBuf][C::NP * TILE];                      // P^T: (n/16)*2048 + (t/8)*128 + (t%8)*16 + n%16
+    uint8_t vt[kVBuf][128 * TILE];                        // V^T: (d/16)*2048 + (t/8)*128 + (t%8)*16 + d%16
+    uint8_t pb[kPBuf][C::NP * TILE];                      // P^T: (n/16)*2048 + (t/8)*128 + (t%8)*16 + n%16
     uint8_t qb[2][C::NS * 128];                       // Q':  (n/8)*1024 + (d/16)*128 + (n%8)*16 + d%16
     uint2 lut[2][128][kLutCopies];
     uint64_t full[kStages], empty[kStages];
-    uint64_t kfull[kBuf], kempty[kBuf], sfull[kBuf], sempty[kBuf], vfull[kBuf], pfull[kBuf], pvdone[kBuf];
+    uint64_t kfull[kKBuf], kempty[kKBuf], vfull[kVBuf], vtfree[kVBuf];
+    uint64_t sfull[kSBuf], sempty[kSBuf], pfull[kPBuf], pvdone[kPBuf];
     uint64_t qfull[2];
     uint64_t mma_done;
     int32_t lens[kMaxBatchPerLaunch];
@@ -307,10 +311,22 @@ __device__ __forceinline__ int tile_valid(const Unit& u, int64_t gt) {
     return v > TILE ? TILE : v;
 }
 
-// Walk over the tiles with work (valid > 0) of a CTA range, in order.
+// Walk over the tiles with work (valid > 0) of a CTA range, in order.  The
+// segment ordinal counts every segment (unit) of the range, empty ones too.
 struct TileWalker {
     int64_t seg_lo, seg_hi, gt, t_end;
     Unit u;
+    int64_t last;                                     // the tile returned by next()
+    int32_t j;                                        // its segment ordinal
+    bool first;                                       // first tile with work of its segment
+    bool fresh;
+
+    __device__ __forceinline__ void start(int64_t t_begin, int64_t t_end_) {
+        seg_lo = seg_hi = gt = t_begin;
+        t_end = t_end_;
+        j = -1;
+        fresh = true;
+    }
     // advance to the next tile with work; false at the end of the range
     __device__ __forceinline__ bool next(const int32_t* prefix, const int32_t* lens, int B, int Hkv) {
         for (;;) {
@@ -318,18 +334,21 @@ struct TileWalker {
                 const int64_t cur = gt++;
                 if (tile_valid(u, cur) > 0) {
                     last = cur;
+                    first = fresh;
+                    fresh = false;
                     return true;
                 }
                 continue;
             }
+            if (seg_hi >= t_end) return false;
             seg_lo = seg_hi;
-            if (seg_lo >= t_end) return false;
             u = find_unit<TILE>(prefix, lens, B, Hkv, seg_lo);
             seg_hi = u.U1 < t_end ? u.U1 : t_end;
             gt = seg_lo;
+            ++j;
+            fresh = true;
         }
     }
-    int64_t last;                                     // the tile returned by next()
 };
 
 // ---------------------------------------------------------------------------
@@ -405,20 +424,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
     }
     // the load warp sets up every barrier and starts the first copies at once
     TileWalker load_walk;
-    load_walk.seg_lo = load_walk.seg_hi = load_walk.gt = t_begin;
-    load_walk.t_end = t_end;
+    load_walk.start(t_begin, t_end);
     uint32_t load_w = 0;
     if (warp == kLoadWarp && lane == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 8);
         }
-        for (int b = 0; b < kBuf; ++b) {
+        for (int b = 0; b < kKBuf; ++b) {
             mbar_init(&sm.kfull[b], 8);
             mbar_init(&sm.kempty[b], 1);
+        }
+        for (int b = 0; b < kVBuf; ++b) {
+            mbar_init(&sm.vfull[b], 8);
+            mbar_init(&sm.vtfree[b], 1);
+        }
+        for (int b = 0; b < kSBuf; ++b) {
             mbar_init(&sm.sfull[b], 1);
             mbar_init(&sm.sempty[b], 4);
-            mbar_init(&sm.vfull[b], 8);
+        }
+        for (int b = 0; b < kPBuf; ++b) {
             mbar_init(&sm.pfull[b], 4);
             mbar_init(&sm.pvdone[b], 1);
         }
@@ -480,65 +505,77 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
         }
     } else if (warp == kMmaWarp) {
         // ================= tensor-core MMAs (one thread) =================
+        // Q.K^T runs ahead of the softmax as far as the S buffers allow; P.V
+        // follows the softmax.  Both streams are polled, so neither waits
+        // behind the other.
         if (lane == 0) {
             const uint32_t idesc_qk = tc::idesc_e4m3(128, NS, false, false, false);
             const uint32_t idesc_pv = tc::idesc_e4m3(128, C::NP, true, true, false);
-            uint32_t w = 0;
-            int64_t pending = -1;                   // work tile whose P.V is still to issue
-            bool pending_first = false;
+            TileWalker qk, pv;
+            qk.start(t_begin, t_end);
+            pv.start(t_begin, t_end);
+            bool qk_more = qk.next(sm.prefix, sm.lens, B, p.Hkv);
+            bool pv_more = pv.next(sm.prefix, sm.lens, B, p.Hkv);
+            uint32_t wq = 0, wp = 0;                   // work tiles issued per stream
+            int32_t q_seg = -1;                        // segment whose query operand is in place
+            uint32_t idle = 0;
             bool ok = true;
-            auto issue_pv = [&](uint32_t v, bool first) {
-                const int b = (int)(v % kBuf);
-                ok = ok && wait_one(&sm.vfull[b], (v / kBuf) & 1u, abort_flag, p.status);
-                ok = ok && wait_one(&sm.pfull[b], (v / kBuf) & 1u, abort_flag, p.status);
-                if (!ok) return;
-                tc::fence_after_sync();
-                const uint32_t va = tc::smem_addr(sm.vt[b]);
-                const uint32_t pa = tc::smem_addr(sm.pb[b]);
+            while (ok && (qk_more || pv_more)) {
+                bool progress = false;
+                if (pv_more && wp < wq) {
+                    const int bv = (int)(wp % kVBuf), bp = (int)(wp % kPBuf);
+                    if (mbar_test_wait(&sm.vfull[bv], (wp / kVBuf) & 1u) &&
+                        mbar_test_wait(&sm.pfull[bp], (wp / kPBuf) & 1u)) {
+                        tc::fence_after_sync();
+                        const uint32_t va = tc::smem_addr(sm.vt[bv]);
+                        const uint32_t pa = tc::smem_addr(sm.pb[bp]);
+                        const bool first = pv.first;   // O restarts with each unit
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_e4m3_ss(tbase + C::COL_O, tc::smem_desc(va + ks * 512, 128, 2048),
-                                    tc::smem_desc(pa + ks * 512, 128, 2048), idesc_pv, !first || ks > 0);
-                tc::mma_commit(&sm.pvdone[b]);
-            };
-            uint32_t j = 0;
-            for (int64_t seg_lo = t_begin; seg_lo < t_end && ok; ++j) {
-                const Unit u = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, seg_lo);
-                const int64_t seg_hi = u.U1 < t_end ? u.U1 : t_end;
-                if (u.L <= 0 && pending >= 0) {
-                    // a unit without tiles: the softmax warps reach its end (and the
-                    // next query operand) only after reading the pending P.V
-                    issue_pv((uint32_t)pending, pending_first);
-                    pending = -1;
+                        for (int ks = 0; ks < 4; ++ks)
+                            tc::mma_e4m3_ss(tbase + C::COL_O, tc::smem_desc(va + ks * 512, 128, 2048),
+                                            tc::smem_desc(pa + ks * 512, 128, 2048), idesc_pv,
+                                            !first || ks > 0);
+                        tc::mma_commit(&sm.pvdone[bp]);
+                        tc::mma_commit(&sm.vtfree[bv]);
+                        ++wp;
+                        pv_more = pv.next(sm.prefix, sm.lens, B, p.Hkv);
+                        progress = true;
+                    }
                 }
-                ok = ok && wait_one(&sm.qfull[j & 1u], (j >> 1) & 1u, abort_flag, p.status);
-                const uint32_t qa = tc::smem_addr(sm.qb[j & 1u]);
-                bool first = true;
-                for (int64_t gt = seg_lo; gt < seg_hi && ok; ++gt) {
-                    if (tile_valid(u, gt) <= 0) continue;
-                    const int b = (int)(w % kBuf);
-                    ok = wait_one(&sm.kfull[b], (w / kBuf) & 1u, abort_flag, p.status);
-                    if (ok && w >= kBuf)
-                        ok = wait_one(&sm.sempty[b], ((w / kBuf) - 1) & 1u, abort_flag, p.status);
-                    if (!ok) break;
-                    tc::fence_after_sync();
-                    const uint32_t kcol = tbase + C::COL_K + 32 * b;
-                    const uint32_t scol = tbase + C::COL_S + NS * b;
+                if (qk_more) {
+                    const int bk = (int)(wq % kKBuf), bs = (int)(wq % kSBuf);
+                    const int32_t jq = qk.j;
+                    const bool q_ok = q_seg == jq || mbar_test_wait(&sm.qfull[jq & 1], (jq >> 1) & 1u);
+                    if (q_ok) q_seg = jq;
+                    if (q_ok && mbar_test_wait(&sm.kfull[bk], (wq / kKBuf) & 1u) &&
+                        (wq < (uint32_t)kSBuf || mbar_test_wait(&sm.sempty[bs], ((wq / kSBuf) - 1) & 1u))) {
+                        tc::fence_after_sync();
+                        const uint32_t qa = tc::smem_addr(sm.qb[jq & 1]);
+                        const uint32_t kcol = tbase + C::COL_K + 32 * bk;
+                        const uint32_t scol = tbase + C::COL_S + NS * bs;
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        tc::mma_e4m3_ts(scol, kcol + 8 * ks, tc::smem_desc(qa + ks * 256, 128, 1024),
-                                        idesc_qk, ks > 0);
-                    tc::mma_commit(&sm.sfull[b]);
-                    tc::mma_commit(&sm.kempty[b]);
-                    if (pending >= 0) issue_pv((uint32_t)pending, pending_first);
-                    pending = w;
-                    pending_first = first;
-                    first = false;
-                    ++w;
+                        for (int ks = 0; ks < 4; ++ks)
+                            tc::mma_e4m3_ts(scol, kcol + 8 * ks, tc::smem_desc(qa + ks * 256, 128, 1024),
+                                            idesc_qk, ks > 0);
+                        tc::mma_commit(&sm.sfull[bs]);
+                        tc::mma_commit(&sm.kempty[bk]);
+                        ++wq;
+                        qk_more = qk.next(sm.prefix, sm.lens, B, p.Hkv);
+                        progress = true;
+                    }
                 }
-                seg_lo = seg_hi;
+                if (progress) {
+                    idle = 0;
+                } else {
+                    if (*reinterpret_cast<volatile int32_t*>(abort_flag)) break;
+                    if (++idle > kMmaIdlePolls) {
+                        atomicExch(abort_flag, 1);
+                        report(p.status, NVFP4_ERR_TIMEOUT);
+                        ok = false;
+                    }
+                    __nanosleep(32);
+                }
             }
-            if (ok && pending >= 0) issue_pv((uint32_t)pending, pending_first);
             // every issued MMA must complete before tensor memory is released
             tc::mma_commit(&sm.mma_done);
             if (!mbar_wait_sleep(&sm.mma_done, 0, kWaitPolls)) report(p.status, NVFP4_ERR_TIMEOUT);
@@ -560,12 +597,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
             for (int64_t gt = seg_lo; gt < seg_hi && ok; ++gt) {
                 if (tile_valid(u, gt) <= 0) continue;
                 const int s = (int)(w % kStages);
-                const int b = (int)(w % kBuf);
+                const int bk = (int)(w % kKBuf), bv = (int)(w % kVBuf);
                 ok = wait_warp(&sm.full[s], (w / kStages) & 1u, abort_flag, p.status);
-                if (ok && w >= kBuf)       // Q.K^T of tile w - kBuf has read this K buffer
-                    ok = wait_warp(&sm.kempty[b], ((w / kBuf) - 1) & 1u, abort_flag, p.status);
-                if (ok && w >= kBuf)       // P.V of tile w - kBuf has read this V^T buffer
-                    ok = wait_warp(&sm.pvdone[b], ((w / kBuf) - 1) & 1u, abort_flag, p.status);
+                if (ok && w >= kKBuf)      // Q.K^T of tile w - kKBuf has read this K buffer
+                    ok = wait_warp(&sm.kempty[bk], ((w / kKBuf) - 1) & 1u, abort_flag, p.status);
                 if (!ok) break;
                 const uint8_t* st = sm.ring[s];
                 uint4 xk[2], xv[2];
@@ -589,9 +624,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
                     dequant_word(xk[j].z, l1.x, l1.y, kf[8 * j + 4], kf[8 * j + 5]);
                     dequant_word(xk[j].w, l1.x, l1.y, kf[8 * j + 6], kf[8 * j + 7]);
                 }
-                tmem_st_x16(trow + C::COL_K + 32 * b + 16 * h, kf);
+                tmem_st_x16(trow + C::COL_K + 32 * bk + 16 * h, kf);
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.kfull[bk]);  // Q.K^T may start before V is done
+                // P.V of tile w - kVBuf has read this V^T buffer
+                if (w >= kVBuf && !wait_warp(&sm.vtfree[bv], ((w / kVBuf) - 1) & 1u, abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
                 // V: 64 codes -> 4 rows of 16 head_dim bytes of V^T
-                uint8_t* dst = sm.vt[b] + (4 * h) * 2048 + (t / 8) * 128 + (t % 8) * 16;
+                uint8_t* dst = sm.vt[bv] + (4 * h) * 2048 + (t / 8) * 128 + (t % 8) * 16;
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int cc = j ^ rot;                // head_dim 64h + 32cc .. +31
@@ -606,13 +650,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
                     *reinterpret_cast<uint4*>(dst + (2 * cc + 1) * 2048) = o1;
                 }
                 fence_proxy_async_smem();
-                tc::tmem_wait_st();
-                tc::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&sm.kfull[b]);
-                    mbar_arrive(&sm.vfull[b]);
-                }
+                if (lane == 0) mbar_arrive(&sm.vfull[bv]);
                 ++w;
             }
             seg_lo = seg_hi;
@@ -651,17 +690,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
             for (int64_t gt = seg_lo; gt < seg_hi; ++gt) {
                 const int valid = tile_valid(u, gt);
                 if (valid <= 0) continue;
-                const int b = (int)(w % kBuf);
+                const int bs = (int)(w % kSBuf), bp = (int)(w % kPBuf);
                 float s[NQ];
-                if (!aborted && !wait_warp(&sm.sfull[b], (w / kBuf) & 1u, abort_flag, p.status)) aborted = true;
+                if (!aborted && !wait_warp(&sm.sfull[bs], (w / kSBuf) & 1u, abort_flag, p.status)) aborted = true;
                 if (!aborted) {
                     tc::fence_after_sync();
                     uint32_t r[NS];
-                    tmem_ld_cols<NS>(trow + C::COL_S + NS * b, r);
+                    tmem_ld_cols<NS>(trow + C::COL_S + NS * bs, r);
                     tc::tmem_wait_ld();
                     tc::fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.sempty[b]);
+                    if (lane == 0) mbar_arrive(&sm.sempty[bs]);
                     const bool live = t < valid;
 #pragma unroll
                     for (int q = 0; q < NQ; ++q)
@@ -698,7 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
                     if (any_pv && !aborted) {
                         // the previous P.V must have landed in O before it is rescaled
                         const uint32_t v = w - 1;
-                        if (!wait_warp(&sm.pvdone[v % kBuf], (v / kBuf) & 1u, abort_flag, p.status)) aborted = true;
+                        if (!wait_warp(&sm.pvdone[v % kPBuf], (v / kPBuf) & 1u, abort_flag, p.status)) aborted = true;
                         if (!aborted) {
                             tc::fence_after_sync();
 #pragma unroll
@@ -730,11 +769,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
 #pragma unroll
                     for (int k = 0; k < NTERM; ++k) tw[k][q / 4] = ta[k] | (tb[k] << 16);
                 }
-                if (!aborted && w >= kBuf &&
-                    !wait_warp(&sm.pvdone[b], ((w / kBuf) - 1) & 1u, abort_flag, p.status))
+                if (!aborted && w >= kPBuf &&
+                    !wait_warp(&sm.pvdone[bp], ((w / kPBuf) - 1) & 1u, abort_flag, p.status))
                     aborted = true;
                 if (!aborted) {
-                    uint8_t* dst = sm.pb[b] + (t / 8) * 128 + (t % 8) * 16;
+                    uint8_t* dst = sm.pb[bp] + (t / 8) * 128 + (t % 8) * 16;
 #pragma unroll
                     for (int k = 0; k < NTERM; ++k) {
                         const int n = k * NQ;
@@ -749,7 +788,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
                     fence_proxy_async_smem();
                     tc::fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.pfull[b]);
+                    if (lane == 0) mbar_arrive(&sm.pfull[bp]);
                 }
                 any_pv = true;
                 ++w;
@@ -769,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
             for (int q = 0; q < NQ; ++q) o[q] = 0.0f;
             if (any_pv && !aborted) {
                 const uint32_t v = w - 1;
-                if (!wait_warp(&sm.pvdone[v % kBuf], (v / kBuf) & 1u, abort_flag, p.status)) aborted = true;
+                if (!wait_warp(&sm.pvdone[v % kPBuf], (v / kPBuf) & 1u, abort_flag, p.status)) aborted = true;
                 if (!aborted) {
                     tc::fence_after_sync();
                     float scale = 1.0f;
