@@ -136,8 +136,8 @@ struct CombineSmem {
 // The partials sit in L2; the merge is written so that every load of a round
 // is independent (one L2 latency per round, not one per contributor):
 // contributors are taken 32 at a time; their (m, l) pairs are fetched by all
-// threads at once into shared memory, and each thread then streams float4
-// slices of the O partials of eight contributors per batch.
+// threads at once into shared memory, and each thread then loads float4
+// slices of the O partials of up to 16 contributors per batch.
 // The merge runs on a group of THREADS threads (tid, warp, lane relative to
 // the group) that synchronizes on named barrier BAR (0: the whole CTA).
 // ---------------------------------------------------------------------------
@@ -148,6 +148,7 @@ __device__ __noinline__ void combine_partials(const Params& p, CombineSmem& cs, 
                                                  int warp, int lane) {
     constexpr int kQ = 8 * NT;                       // g <= kQ
     constexpr int kOut4 = (kQ * D / 4 + THREADS - 1) / THREADS;   // float4 outputs per thread
+    constexpr int kBatch = kOut4 >= 4 ? 4 : 16 / kOut4;          // contributors per batch of loads
     const int g = p.g;
     const int n4 = g * D / 4;                        // float4 outputs of the unit
     const int ncc = (int)(c_last - c_first + 1);
@@ -211,32 +212,32 @@ __device__ __noinline__ void combine_partials(const Params& p, CombineSmem& cs, 
         }
         group_sync<THREADS, BAR>();
         const int nj = ncc - base < 32 ? ncc - base : 32;
-        for (int j0 = 0; j0 < nj; j0 += 8) {
+        for (int j0 = 0; j0 < nj; j0 += kBatch) {
+            float4 v[kOut4][kBatch];
+            float w[kOut4][kBatch];
 #pragma unroll
-            for (int k = 0; k < kOut4; ++k) {
+            for (int k = 0; k < kOut4; ++k) {          // every load of the batch in flight at once
                 const int i4 = tid + k * THREADS;
-                if (i4 < n4) {
-                    const int q = (i4 * 4) / D;
-                    float4 v[8];
-                    float w[8];
+                const int q = i4 < n4 ? (i4 * 4) / D : 0;
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) {      // eight independent loads in flight
-                        const int j = j0 + jj;
-                        const int sl = j < nj ? cs.slot[j] : -1;
-                        w[jj] = sl >= 0 ? cs.l[q][j] : 0.0f;
-                        v[jj] = sl >= 0 ? __ldcg(reinterpret_cast<const float4*>(
-                                              p.partials + (int64_t)sl * slot_floats) + i4)
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-#pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) {
-                        acc[k].x = fmaf(w[jj], v[jj].x, acc[k].x);
-                        acc[k].y = fmaf(w[jj], v[jj].y, acc[k].y);
-                        acc[k].z = fmaf(w[jj], v[jj].z, acc[k].z);
-                        acc[k].w = fmaf(w[jj], v[jj].w, acc[k].w);
-                    }
+                for (int jj = 0; jj < kBatch; ++jj) {
+                    const int j = j0 + jj;
+                    const int sl = (j < nj && i4 < n4) ? cs.slot[j] : -1;
+                    w[k][jj] = sl >= 0 ? cs.l[q][j] : 0.0f;
+                    v[k][jj] = sl >= 0 ? __ldcg(reinterpret_cast<const float4*>(
+                                             p.partials + (int64_t)sl * slot_floats) + i4)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
+#pragma unroll
+            for (int k = 0; k < kOut4; ++k)
+#pragma unroll
+                for (int jj = 0; jj < kBatch; ++jj) {
+                    acc[k].x = fmaf(w[k][jj], v[k][jj].x, acc[k].x);
+                    acc[k].y = fmaf(w[k][jj], v[k][jj].y, acc[k].y);
+                    acc[k].z = fmaf(w[k][jj], v[k][jj].z, acc[k].z);
+                    acc[k].w = fmaf(w[k][jj], v[k][jj].w, acc[k].w);
+                }
         }
     }
     group_sync<THREADS, BAR>();

@@ -102,6 +102,8 @@ struct __align__(1024) Smem {
     CombineSmem comb;
     uint32_t tmem_base;
     int32_t last_flag;
+    int32_t n_pend;                                   // units this CTA must merge at its end
+    int64_t pend_gt[2];
     int32_t abort_flag;
 };
 
@@ -452,7 +454,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
         mbar_init(&sm.mma_done, 1);
         fence_mbar_init();
         sm.abort_flag = 0;
-        while (load_w < (uint32_t)kStages && load_walk.next(sm.prefix, sm.lens, B, p.Hkv)) {
+        sm.n_pend = 0;
+        // the first two tiles only: the CTA barrier below waits for this lane
+        while (load_w < 2u && load_walk.next(sm.prefix, sm.lens, B, p.Hkv)) {
             issue_tile<128, TILE>(p, load_walk.u, load_walk.last, sm.ring[load_w], &sm.full[load_w]);
             ++load_w;
         }
@@ -490,7 +494,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
             uint32_t w = load_w;                       // the first stages went out in the prologue
             while (load_walk.next(sm.prefix, sm.lens, B, p.Hkv)) {
                 const int s = (int)(w % kStages);
-                if (!wait_one(&sm.empty[s], ((w / kStages) - 1) & 1u, abort_flag, p.status)) break;
+                if (w >= (uint32_t)kStages && !wait_one(&sm.empty[s], ((w / kStages) - 1) & 1u, abort_flag, p.status))
+                    break;
                 issue_tile<128, TILE>(p, load_walk.u, load_walk.last, sm.ring[s], &sm.full[s]);
                 ++w;
             }
@@ -871,12 +876,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
                     sm.last_flag = (prev == contributors - 1);
                 }
                 softmax_sync();
-                if (sm.last_flag) {
-                    __threadfence();
-                    combine_partials<128, NT, 128, kSoftmaxBar>(p, sm.comb, u, T, N, c_first, c_last,
-                                                               slot_floats, t, sw, lane);
-                    if (t == 0) atomicExch(&p.counters[(int64_t)u.b * p.Hkv + u.h], 0);
-                }
+                // the merge waits until every role of this CTA is done and then
+                // runs on all its threads (a CTA is last for at most two units)
+                if (sm.last_flag && t == 0) sm.pend_gt[sm.n_pend++] = u.U0;
             }
             softmax_sync();
             seg_lo = seg_hi;
@@ -888,6 +890,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
     __syncthreads();
     tc::fence_after_sync();
     if (warp == kMmaWarp) tc::tmem_dealloc(tbase, C::kTmemCols);
+
+    // ---- split-K merges of the units this CTA finished last, on every thread ----
+    const int n_pend = sm.n_pend;
+    for (int i = 0; i < n_pend; ++i) {
+        const Unit u = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, sm.pend_gt[i]);
+        __threadfence();
+        combine_partials<128, NT, kThreads, 0>(p, sm.comb, u, T, N, cta_of(u.U0, T, N),
+                                               cta_of(u.U1 - 1, T, N), partial_slot_floats(p.g, 128),
+                                               tid, warp, lane);
+        if (tid == 0) atomicExch(&p.counters[(int64_t)u.b * p.Hkv + u.h], 0);
+    }
 }
 
 template <int NT>
