@@ -43,7 +43,9 @@ METRIC = "NVFP4 decode-attention KV-tokens/s and achieved HBM GB/s (% of peak) a
 UNIT = "KV-tokens/s"
 DTYPE = "nvfp4 (e2m1 + e4m3 block scale) storage, fp8 e4m3 values, f16 MMA inputs, f32 accumulate"
 FALLBACK_HBM_GBS = 6650.0
-ATTN_SOURCES = ["bit_decode_attention_b200/csrc/nvfp4kv_decode_attention.cu",
+ATTN_SOURCES = ["bit_decode_attention_b200/csrc/nvfp4kv_decode_attention_tc.cu",
+                "bit_decode_attention_b200/csrc/nvfp4kv_attention_common.cuh",
+                "bit_decode_attention_b200/csrc/nvfp4kv_tcgen05.cuh",
                 "bit_decode_attention_b200/csrc/nvfp4kv_device.cuh"]
 
 
@@ -530,7 +532,8 @@ def main():
                 "frac": achieved / peak, "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback",
                 "traffic": profiled_traffic("decode_attention_%s_traffic.json" % w.name),
-                "kernel": "decode_attention_kernel<128,1,false>",
+                "kernel": "decode_attention_tc_kernel<%d> (tcgen05, head_dim 128, bf16 queries)"
+                          % (1 if w.Hq // w.Hkv <= 8 else 2),
                 "algorithmic_bytes_per_launch": wl.attention_bytes(),
                 "launch_ms": att_ms, "launches_sampled": att_n,
                 "frac_of_nominal_8tbs": achieved / 8000.0}
