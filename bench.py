@@ -227,10 +227,10 @@ class DecodeWorkload:
         torch.cuda.synchronize()
         assert self.status.item() == 0, "device status %d during set-up" % self.status.item()
 
-    # kernels per step (ours): 2 appends + 1 attention
+    # kernels per step (ours): 1 append of K and V + 1 attention
     @property
     def launches_per_step(self):
-        return 3 if self.with_append else 1
+        return 2 if self.with_append else 1
 
     def tokens_per_step(self):
         return self.w.B * self.L_att
@@ -246,8 +246,8 @@ class DecodeWorkload:
     def step(self, j, events=None):
         nv, r = self.nv, j % self.R
         if self.with_append:
-            nv.nvfp4_kv_quantize_append(self.new_k[r], self.start, self.sk, self.k[r], status=self.status)
-            nv.nvfp4_kv_quantize_append(self.new_v[r], self.start, self.sv, self.v[r], status=self.status)
+            nv.nvfp4_kv_quantize_append_kv(self.new_k[r], self.new_v[r], self.start, self.sk, self.sv,
+                                           self.k[r], self.v[r], status=self.status)
         if events is not None:
             events[0].record()
         nv.nvfp4_decode_attention(self.q[r], self.k[r], self.v[r], self.sk, self.sv, self.lens,
@@ -334,8 +334,8 @@ def time_e2e(wl, steps):
         d_k[r].copy_(h_k[r], non_blocking=True)
         d_v[r].copy_(h_v[r], non_blocking=True)
         d_q[r].copy_(h_q[r], non_blocking=True)
-        nv.nvfp4_kv_quantize_append(d_k[r], wl.start, wl.sk, wl.k[r], status=wl.status)
-        nv.nvfp4_kv_quantize_append(d_v[r], wl.start, wl.sv, wl.v[r], status=wl.status)
+        nv.nvfp4_kv_quantize_append_kv(d_k[r], d_v[r], wl.start, wl.sk, wl.sv, wl.k[r], wl.v[r],
+                                       status=wl.status)
         nv.nvfp4_decode_attention(d_q[r], wl.k[r], wl.v[r], wl.sk, wl.sv, wl.lens, out=wl.out[r],
                                   workspace=wl.ws, status=wl.status)
         h_out[r].copy_(wl.out[r], non_blocking=True)

@@ -24,6 +24,7 @@ from ._native import (NVFP4_ERR_CAPACITY, NVFP4_ERR_INVALID_ARG, NVFP4_ERR_NONFI
 
 __all__ = [
     "KVPlane", "nvfp4_cache_bytes", "nvfp4_calib_tensor_scale", "nvfp4_kv_quantize_append",
+    "nvfp4_kv_quantize_append_kv",
     "nvfp4_kv_dequant_fp8", "nvfp4_decode_attention_workspace", "nvfp4_decode_attention",
     "nvfp4_version", "NativeError", "nvfp4_decode_attention_noalloc",
 ]
@@ -109,6 +110,23 @@ def nvfp4_kv_quantize_append(x_new: torch.Tensor, start_pos: torch.Tensor, s_ten
                                                 _ptr(start_pos), _ptr(new_lens), _ptr(s_tensor),
                                                 ctypes.byref(pl), _ptr(status), _stream(stream))
     _native.check("nvfp4_kv_quantize_append", st)
+
+
+def nvfp4_kv_quantize_append_kv(x_k: torch.Tensor, x_v: torch.Tensor, start_pos: torch.Tensor,
+                                s_tensor_k: torch.Tensor, s_tensor_v: torch.Tensor, k: KVPlane, v: KVPlane,
+                                new_lens: Optional[torch.Tensor] = None,
+                                status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """nvfp4_kv_quantize_append for K into `k` and V into `v` in one launch."""
+    _need_cuda(x_k, x_v, start_pos, s_tensor_k, s_tensor_v, new_lens, status)
+    if x_k.shape != x_v.shape or x_k.dtype != x_v.dtype:
+        raise ValueError("x_k and x_v must have the same shape and dtype")
+    n_new = x_k.shape[1]
+    pk, pv = k.struct(), v.struct()
+    st = _native.lib().nvfp4_kv_quantize_append_kv(_ptr(x_k), _ptr(x_v), _dtype_code(x_k), n_new,
+                                                   _ptr(start_pos), _ptr(new_lens), _ptr(s_tensor_k),
+                                                   _ptr(s_tensor_v), ctypes.byref(pk), ctypes.byref(pv),
+                                                   _ptr(status), _stream(stream))
+    _native.check("nvfp4_kv_quantize_append_kv", st)
 
 
 def nvfp4_kv_dequant_fp8(plane: KVPlane, s_tensor: torch.Tensor, seq_lens: torch.Tensor,

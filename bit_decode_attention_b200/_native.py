@@ -29,6 +29,7 @@ EXPORTS = (
     "nvfp4_cache_bytes",
     "nvfp4_calib_tensor_scale",
     "nvfp4_kv_quantize_append",
+    "nvfp4_kv_quantize_append_kv",
     "nvfp4_kv_dequant_fp8",
     "nvfp4_decode_attention_workspace",
     "nvfp4_decode_attention",
@@ -78,6 +79,8 @@ def lib():
     L.nvfp4_calib_tensor_scale.restype = i32
     L.nvfp4_kv_quantize_append.argtypes = [vp, i32, i32, vp, vp, vp, plane_p, vp, vp]
     L.nvfp4_kv_quantize_append.restype = i32
+    L.nvfp4_kv_quantize_append_kv.argtypes = [vp, vp, i32, i32, vp, vp, vp, vp, plane_p, plane_p, vp, vp]
+    L.nvfp4_kv_quantize_append_kv.restype = i32
     L.nvfp4_kv_dequant_fp8.argtypes = [plane_p, vp, vp, vp, vp, vp]
     L.nvfp4_kv_dequant_fp8.restype = i32
     L.nvfp4_decode_attention_workspace.argtypes = [i32, i32, i32, i32]

@@ -105,6 +105,25 @@ nvfp4_status nvfp4_kv_quantize_append(const void* x_new, nvfp4_dtype dtype, int 
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
+nvfp4_status nvfp4_kv_quantize_append_kv(const void* x_k, const void* x_v, nvfp4_dtype dtype,
+                                         int n_new, const int32_t* d_start_pos, int32_t* d_new_lens,
+                                         const float* d_s_tensor_k, const float* d_s_tensor_v,
+                                         const nvfp4_kv_plane* k, const nvfp4_kv_plane* v,
+                                         int32_t* d_status, nvfp4_stream_t stream) {
+    if (!plane_ok(k) || !plane_ok(v) || n_new < 0 || d_s_tensor_k == nullptr ||
+        d_s_tensor_v == nullptr || d_start_pos == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (k->B != v->B || k->H_kv != v->H_kv || k->S_max != v->S_max || k->D != v->D)
+        return NVFP4_ERR_INVALID_ARG;
+    if (dtype != NVFP4_IN_BF16 && dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
+    if (d_new_lens != nullptr && d_new_lens == d_start_pos) return NVFP4_ERR_INVALID_ARG;
+    if (n_new == 0 || k->B == 0) return NVFP4_OK;
+    if (x_k == nullptr || x_v == nullptr || !aligned16(x_k) || !aligned16(x_v)) return NVFP4_ERR_INVALID_ARG;
+    return from_cuda(launch_quantize_append_kv(x_k, x_v, dtype == NVFP4_IN_F32, n_new, d_start_pos,
+                                               d_new_lens, d_s_tensor_k, d_s_tensor_v, *k, *v,
+                                               d_status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 nvfp4_status nvfp4_kv_dequant_fp8(const nvfp4_kv_plane* plane, const float* d_s_tensor,
                                   const int32_t* d_seq_lens, uint8_t* out_e4m3, int32_t* d_status,
                                   nvfp4_stream_t stream) {

@@ -148,6 +148,69 @@ __device__ __forceinline__ uint32_t quantize_block(const float (&v)[16], float s
     return sb;
 }
 
+// Quantize-append of one plane (a1-a4); `item` enumerates (b, t, h, blk)
+// with blk fastest.  Index math in 32 bits when the item count fits.
+template <bool F32, typename I>
+__device__ __forceinline__ void quantize_append_item(
+    const void* __restrict__ x_new, I i, int B, int n_new, int Hkv, int D,
+    const int32_t* __restrict__ start_pos, int32_t* __restrict__ new_lens, float st, bool st_ok,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int S_max, int32_t* __restrict__ status) {
+    const int nblk = D / 16;
+    const int blk = (int)(i % nblk);
+    I r = i / nblk;
+    const int t = (int)(r % n_new);
+    r /= n_new;
+    const int h = (int)(r % Hkv);
+    const int b = (int)(r / Hkv);
+    const bool leader = (t == 0 && h == 0 && blk == 0);
+    if (!st_ok) {
+        if (i == 0) report(status, NVFP4_ERR_NONFINITE);
+        return;
+    }
+    const int start = start_pos[b];
+    if (start < 0 || (int64_t)start + n_new > S_max) {
+        if (leader) report(status, NVFP4_ERR_CAPACITY);
+        return;
+    }
+    if (leader && new_lens != nullptr) new_lens[b] = start + n_new;
+    float v[16];
+    load16<F32>(x_new, (((int64_t)b * n_new + t) * Hkv + h) * D + 16 * blk, v);
+    uint2 packed;
+    const uint32_t sb = quantize_block(v, st, packed);
+    const int64_t slot = ((int64_t)b * Hkv + h) * S_max + start + t;
+    *reinterpret_cast<uint2*>(codes + slot * (D / 2) + 8 * blk) = packed;
+    scales[slot * (D / 16) + blk] = (uint8_t)sb;
+}
+
+// One launch for the K and V planes of the same tokens: blockIdx.y selects the
+// plane (0: K, which also writes new_lens; 1: V).
+template <bool F32>
+__global__ void __launch_bounds__(256) quantize_append_kv_kernel(
+    const void* __restrict__ x_k, const void* __restrict__ x_v, int B, int n_new, int Hkv, int D,
+    const int32_t* __restrict__ start_pos, int32_t* __restrict__ new_lens,
+    const float* __restrict__ st_k_p, const float* __restrict__ st_v_p,
+    uint8_t* __restrict__ codes_k, uint8_t* __restrict__ scales_k, uint8_t* __restrict__ codes_v,
+    uint8_t* __restrict__ scales_v, int S_max, int32_t* __restrict__ status) {
+    const bool is_v = blockIdx.y == 1;
+    const float st = *(is_v ? st_v_p : st_k_p);
+    const bool st_ok = st > 0.0f && st <= 3.4028234663852886e38f;  // finite and positive
+    const int64_t total = (int64_t)B * Hkv * n_new * (D / 16);
+    const void* x = is_v ? x_v : x_k;
+    uint8_t* codes = is_v ? codes_v : codes_k;
+    uint8_t* scales = is_v ? scales_v : scales_k;
+    int32_t* nl = is_v ? nullptr : new_lens;
+    if (total < (int64_t)INT32_MAX) {
+        for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < (int)total; i += gridDim.x * blockDim.x)
+            quantize_append_item<F32, int>(x, i, B, n_new, Hkv, D, start_pos, nl, st, st_ok, codes, scales,
+                                           S_max, status);
+    } else {
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+             i += (int64_t)gridDim.x * blockDim.x)
+            quantize_append_item<F32, int64_t>(x, i, B, n_new, Hkv, D, start_pos, nl, st, st_ok, codes,
+                                               scales, S_max, status);
+    }
+}
+
 template <bool F32>
 __global__ void __launch_bounds__(256) quantize_append_kernel(
     const void* __restrict__ x_new, int B, int n_new, int Hkv, int D,
@@ -185,6 +248,29 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(
         *reinterpret_cast<uint2*>(codes + slot * (D / 2) + 8 * blk) = packed;
         scales[slot * (D / 16) + blk] = (uint8_t)sb;
     }
+}
+
+cudaError_t launch_quantize_append_kv(const void* x_k, const void* x_v, bool f32, int n_new,
+                                      const int32_t* d_start_pos, int32_t* d_new_lens,
+                                      const float* d_st_k, const float* d_st_v,
+                                      const nvfp4_kv_plane& pk, const nvfp4_kv_plane& pv,
+                                      int32_t* d_status, cudaStream_t stream) {
+    const int64_t total = (int64_t)pk.B * pk.H_kv * n_new * (pk.D / 16);
+    if (total == 0) return cudaSuccess;
+    const int threads = 256;
+    int64_t grid = (total + threads - 1) / threads;
+    const int64_t cap = 8L * device_sm_count();
+    if (grid > cap) grid = cap;
+    const dim3 g((unsigned)grid, 2);
+    if (f32)
+        quantize_append_kv_kernel<true><<<g, threads, 0, stream>>>(
+            x_k, x_v, pk.B, n_new, pk.H_kv, pk.D, d_start_pos, d_new_lens, d_st_k, d_st_v, pk.codes,
+            pk.scales, pv.codes, pv.scales, pk.S_max, d_status);
+    else
+        quantize_append_kv_kernel<false><<<g, threads, 0, stream>>>(
+            x_k, x_v, pk.B, n_new, pk.H_kv, pk.D, d_start_pos, d_new_lens, d_st_k, d_st_v, pk.codes,
+            pk.scales, pv.codes, pv.scales, pk.S_max, d_status);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_append(const void* x_new, bool f32, int n_new,

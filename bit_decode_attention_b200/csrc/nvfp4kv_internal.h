@@ -35,6 +35,12 @@ cudaError_t launch_quantize_append(const void* x_new, bool f32, int n_new,
                                    const float* d_s_tensor, const nvfp4_kv_plane& plane,
                                    int32_t* d_status, cudaStream_t stream);
 
+cudaError_t launch_quantize_append_kv(const void* x_k, const void* x_v, bool f32, int n_new,
+                                      const int32_t* d_start_pos, int32_t* d_new_lens,
+                                      const float* d_st_k, const float* d_st_v,
+                                      const nvfp4_kv_plane& pk, const nvfp4_kv_plane& pv,
+                                      int32_t* d_status, cudaStream_t stream);
+
 cudaError_t launch_dequant_fp8(const nvfp4_kv_plane& plane, const float* d_s_tensor,
                                const int32_t* d_seq_lens, uint8_t* out, int32_t* d_status,
                                cudaStream_t stream);

@@ -136,6 +136,18 @@ nvfp4_status nvfp4_kv_quantize_append(const void* x_new, nvfp4_dtype dtype, int 
                                       const float* d_s_tensor, const nvfp4_kv_plane* plane,
                                       int32_t* d_status, nvfp4_stream_t stream);
 
+/* Quantize-append the same new tokens into the K and the V plane in one
+ * launch ([NVFP4-KV] "量子化・逆量子化フロー": K and V are both quantized
+ * on append).  Same results, arguments and errors as two calls of
+ * nvfp4_kv_quantize_append (K with d_s_tensor_k into k, V with d_s_tensor_v
+ * into v); the planes must agree in B, H_kv, S_max and D.  d_new_lens, if
+ * given, is written once. */
+nvfp4_status nvfp4_kv_quantize_append_kv(const void* x_k, const void* x_v, nvfp4_dtype dtype,
+                                         int n_new, const int32_t* d_start_pos, int32_t* d_new_lens,
+                                         const float* d_s_tensor_k, const float* d_s_tensor_v,
+                                         const nvfp4_kv_plane* k, const nvfp4_kv_plane* v,
+                                         int32_t* d_status, nvfp4_stream_t stream);
+
 /* Dequantize a plane to FP8 E4M3 bytes ([NVFP4-KV] "量子化・逆量子化フロー":
  * NVFP4 -> FP8 before attention).
  *   d_seq_lens device int32 [B]; only slots t < seq_lens[b] are written

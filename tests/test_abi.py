@@ -83,6 +83,13 @@ def test_argument_validation_without_gpu(lib):
     assert qa(dev, 0, 1, dev, dev, dev, ctypes.byref(p), None, None) == INVALID    # aliasing
     assert qa(ctypes.c_void_p(72), 0, 1, dev, None, dev, ctypes.byref(p), None, None) == INVALID
     assert qa(dev, 0, 0, dev, None, dev, ctypes.byref(p), None, None) == 0         # no-op
+    qkv = lib.nvfp4_kv_quantize_append_kv
+    kv_other = _plane(S=32)
+    assert qkv(dev, dev, 0, 1, dev, None, dev, dev, ctypes.byref(p), ctypes.byref(kv_other), None, None) == INVALID
+    assert qkv(dev, dev, 0, 1, dev, None, None, dev, ctypes.byref(p), ctypes.byref(p), None, None) == INVALID
+    assert qkv(dev, ctypes.c_void_p(72), 0, 1, dev, None, dev, dev, ctypes.byref(p), ctypes.byref(p),
+               None, None) == INVALID                                                  # V misaligned
+    assert qkv(dev, dev, 0, 0, dev, None, dev, dev, ctypes.byref(p), ctypes.byref(p), None, None) == 0
     dq = lib.nvfp4_kv_dequant_fp8
     assert dq(ctypes.byref(p), None, dev, dev, None, None) == INVALID
     assert dq(ctypes.byref(p), dev, dev, ctypes.c_void_p(65), None, None) == INVALID

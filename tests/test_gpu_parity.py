@@ -236,3 +236,43 @@ def test_attention_ignores_bytes_past_the_sequence(nv, D, q_dtype):
     got = c.gpu_attention().cpu().numpy()
     assert c.status.item() == 0
     assert_attention_close(got, c.oracle_attention())
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_quantize_append_kv_matches_two_calls(nv, dtype):
+    # one launch for K and V gives the same planes (and new lengths) as two calls,
+    # and both match the oracle
+    w = synthetic.shrink(synthetic.get("gqa"), B=3, Hq=8, Hkv=2, dtype=dtype)
+    n_new = 37
+    xk = synthetic.kv_tokens(w, n_new, "k")
+    xv = synthetic.kv_tokens(w, n_new, "v")
+    start = torch.tensor([0, 5, 100], dtype=torch.int32, device="cuda")
+    S_max = synthetic.capacity(100 + n_new)
+    sk = nv.nvfp4_calib_tensor_scale(to_dev(xk.reshape(-1), dtype))
+    sv = nv.nvfp4_calib_tensor_scale(to_dev(xv.reshape(-1), dtype))
+    xk_d, xv_d = to_dev(xk, dtype), to_dev(xv, dtype)
+    planes = [nv.KVPlane.allocate(w.B, w.Hkv, S_max, w.D) for _ in range(4)]
+    lens_a = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+    lens_b = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_kv_quantize_append_kv(xk_d, xv_d, start, sk, sv, planes[0], planes[1], new_lens=lens_a,
+                                   status=status)
+    nv.nvfp4_kv_quantize_append(xk_d, start, sk, planes[2], new_lens=lens_b, status=status)
+    nv.nvfp4_kv_quantize_append(xv_d, start, sv, planes[3], status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    for a, b in ((planes[0], planes[2]), (planes[1], planes[3])):
+        assert torch.equal(a.codes, b.codes) and torch.equal(a.scales, b.scales)
+    assert lens_a.tolist() == [n_new, 5 + n_new, 100 + n_new] == lens_b.tolist()
+    # oracle: sequence 1, K and V, with the oracle's own tensor scales (equal to the
+    # device's bit for bit, which test_calib_bit_exact covers)
+    rc_k, st_k_o = oracle.tensor_scale(xk.reshape(-1).numpy())
+    rc_v, st_v_o = oracle.tensor_scale(xv.reshape(-1).numpy())
+    assert rc_k == 0 and rc_v == 0
+    assert np.float32(sk.item()).view(np.uint32) == st_k_o.view(np.uint32)
+    assert np.float32(sv.item()).view(np.uint32) == st_v_o.view(np.uint32)
+    for x, st_o, pl in ((xk, st_k_o, planes[0]), (xv, st_v_o, planes[1])):
+        oc, os_ = oracle.new_planes(1, w.Hkv, S_max, w.D)
+        assert oracle.quantize_append(x[1:2].numpy(), np.array([5], np.int32), st_o, oc, os_) == 0
+        np.testing.assert_array_equal(pl.codes[1].cpu().numpy(), oc[0])
+        np.testing.assert_array_equal(pl.scales[1].cpu().numpy(), os_[0])
