@@ -60,9 +60,7 @@ struct Geometry {
     static constexpr int SB = D / 16;                // scale bytes per token
     static constexpr int KS = D / 16;                // k-steps of Q.K^T = m-tiles of P.V
     static constexpr int EK = D / 4;                 // K elements per lane per token
-    static constexpr int WK = EK / 8;                // K code words per lane per token
     static constexpr int EV = D / 8;                 // V channels per lane
-    static constexpr int WV = EV / 8;                // V code words per lane per token
     static constexpr int STAGE = kTile * (2 * KB + 2 * SB);
     static constexpr int OFF_VC = kTile * KB;
     static constexpr int OFF_KS = 2 * kTile * KB;
