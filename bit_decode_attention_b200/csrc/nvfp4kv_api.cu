@@ -159,6 +159,11 @@ nvfp4_status nvfp4_decode_attention(const void* q, nvfp4_dtype q_dtype, int H_q,
     const int B = k->B;
     if (B == 0) return NVFP4_OK;
     if (q == nullptr || out == nullptr || !aligned16(q) || !aligned16(out)) return NVFP4_ERR_INVALID_ARG;
+    // the kernels split a launch's tiles (32 tokens at the smallest) of every
+    // (sequence, KV head) with 32-bit prefix sums
+    const int64_t launch_tiles = (int64_t)(B < kMaxBatchPerLaunch ? B : kMaxBatchPerLaunch) * k->H_kv *
+                                 (((int64_t)k->S_max + 31) / 32);
+    if (launch_tiles > (int64_t)INT32_MAX) return NVFP4_ERR_UNSUPPORTED;
     const AttnWorkspace ws = attention_workspace(B, H_q, k->H_kv, k->D);
     if (workspace == nullptr || workspace_bytes < ws.total_bytes || !aligned16(workspace))
         return NVFP4_ERR_WORKSPACE;

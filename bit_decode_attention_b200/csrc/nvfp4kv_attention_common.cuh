@@ -120,125 +120,167 @@ __device__ __forceinline__ void group_sync() {
 
 // scratch of the split-K merge (see combine_partials)
 struct CombineSmem {
-    int32_t slot[32];         // partial slot of chunk contributor j, -1 if none
-    float m[16][32];          // running max m_j of contributor j for query q
-    float l[16][32];          // l_j, then w_j = 2^(m_j - M) once M is known
-    float M[16];
-    float L[16];
+    float w[16][32];          // w_j = 2^(m_j - M) of chunk contributor j for query q
+    float L[16];              // sum_j w_j l_j over every contributor
 };
+
+// Number of CTAs holding a partial of the unit of global tiles [U0, U1).
+// With T >= N every range is non-empty, so each CTA from cta_of(U0) to
+// cta_of(U1 - 1) holds one; with T < N a non-empty range is a single tile,
+// so there is one CTA per tile.  (No loop over CTAs: a 64-bit division costs
+// a few hundred cycles, and the count sits on the critical path of the merge.)
+__device__ __forceinline__ int unit_contributors(int64_t U0, int64_t U1, int64_t T, int64_t N) {
+    return T >= N ? (int)(cta_of(U1 - 1, T, N) - cta_of(U0, T, N) + 1) : (int)(U1 - U0);
+}
+
+// Count one CTA's arrival at a split unit.  The CTA's partial stores are
+// ordered before this by a CTA barrier; the release half of the atomic
+// publishes them (it is cumulative over the barrier), and its acquire half
+// makes the other contributors' stores visible to a CTA that arrives last,
+// once a second CTA barrier follows.  One atomic per CTA replaces a fence on
+// every thread: a sequentially consistent GPU fence costs about a
+// microsecond, and they do not overlap.
+__device__ __forceinline__ int arrive_split_unit(int32_t* counter) {
+    int prev;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(prev) : "l"(counter) : "memory");
+    return prev;
+}
 
 // ---------------------------------------------------------------------------
 // Split-K merge of one (sequence, KV head) unit by the last CTA to finish with
-// it.  The contributors are CTAs c_first..c_last (those with non-empty ranges);
-// each left (m, l, O) per query in its partial slot.  Out = sum_c w_c O_c /
-// sum_c w_c l_c with w_c = 2^(m_c - M), M = max_c m_c.
+// it.  Contributor j (0 <= j < unit_contributors) left (m, l, O) per query in
+// its partial slot.  Out = sum_j w_j O_j / sum_j w_j l_j with
+// w_j = 2^(m_j - M), M = max_j m_j.
 //
-// The partials sit in L2; the merge is written so that every load of a round
-// is independent (one L2 latency per round, not one per contributor):
-// contributors are taken 32 at a time; their (m, l) pairs are fetched by all
-// threads at once into shared memory, and each thread then loads float4
-// slices of the O partials of up to 16 contributors per batch.
+// The partials sit in L2, so the merge is a handful of L2 round trips:
+// every thread issues its float4 loads of the first batch of O partials at
+// once, together with the (m, l) loads (warp q, lane j: query q of
+// contributor j), and only then waits.  Contributors are taken 32 at a time
+// (one lane each); a thread keeps up to 16 O loads in flight.
 // The merge runs on a group of THREADS threads (tid, warp, lane relative to
 // the group) that synchronizes on named barrier BAR (0: the whole CTA).
 // ---------------------------------------------------------------------------
 template <int D, int NT, int THREADS, int BAR = 0>
 __device__ __noinline__ void combine_partials(const Params& p, CombineSmem& cs, const Unit& u,
-                                                 int64_t T, int64_t N, int64_t c_first,
-                                                 int64_t c_last, int64_t slot_floats, int tid,
+                                                 int64_t T, int64_t N, int64_t slot_floats, int tid,
                                                  int warp, int lane) {
-    constexpr int kQ = 8 * NT;                       // g <= kQ
+    constexpr int kQ = 8 * NT;                                    // g <= kQ
+    constexpr int kWarps = THREADS / 32;
+    constexpr int kQW = (kQ + kWarps - 1) / kWarps;               // queries per warp
     constexpr int kOut4 = (kQ * D / 4 + THREADS - 1) / THREADS;   // float4 outputs per thread
     constexpr int kBatch = kOut4 >= 4 ? 4 : 16 / kOut4;          // contributors per batch of loads
     const int g = p.g;
     const int n4 = g * D / 4;                        // float4 outputs of the unit
-    const int ncc = (int)(c_last - c_first + 1);
+    const bool dense = T >= N;                       // every CTA range non-empty
+    const int64_t c_first = cta_of(u.U0, T, N);
+    const int ncc = unit_contributors(u.U0, u.U1, T, N);
+    // the first contributor's slot is odd when the unit starts inside its range
+    const bool first_odd = range_start(c_first, T, N) < u.U0;
+    auto part_of = [&](int j) -> const float* {
+        const int64_t cc = dense ? c_first + j : cta_of(u.U0 + j, T, N);
+        return p.partials + (2 * cc + ((j == 0 && first_odd) ? 1 : 0)) * slot_floats;
+    };
     float4 acc[kOut4];
+    float4 v[kOut4][kBatch];
 #pragma unroll
     for (int k = 0; k < kOut4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (tid < kQ) {
-        cs.M[tid] = -INFINITY;
-        cs.L[tid] = 0.0f;
-    }
-    // one chunk of up to 32 contributors: slots, then (m, l) of every query
-    auto load_chunk = [&](int base) {
-        group_sync<THREADS, BAR>();
-        if (warp == 0) {
-            int sl = -1;
-            if (base + lane < ncc) {
-                const int64_t cc = c_first + base + lane;
-                if (range_start(cc, T, N) < range_start(cc + 1, T, N))
-                    sl = (int)partial_slot(cc, u.U0, T, N);
+    // O loads of contributors j0 .. j0 + kBatch - 1 (those below jlim)
+    auto issue = [&](int j0, int jlim) {
+#pragma unroll
+        for (int k = 0; k < kOut4; ++k) {
+            const int i4 = tid + k * THREADS;
+#pragma unroll
+            for (int jj = 0; jj < kBatch; ++jj) {
+                const int j = j0 + jj;
+                v[k][jj] = (j < jlim && i4 < n4)
+                               ? __ldcg(reinterpret_cast<const float4*>(part_of(j)) + i4)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            cs.slot[lane] = sl;
         }
-        group_sync<THREADS, BAR>();
-        for (int i = tid; i < 32 * kQ; i += THREADS) {
-            const int j = i & 31, q = i >> 5;
-            const int sl = cs.slot[j];
-            float m = -INFINITY, l = 0.0f;
-            if (sl >= 0 && q < g) {
-                const float* part = p.partials + (int64_t)sl * slot_floats;
-                m = __ldcg(part + g * D + q);
-                l = __ldcg(part + g * D + g + q);
-            }
-            cs.m[q][j] = m;
-            cs.l[q][j] = l;
-        }
-        group_sync<THREADS, BAR>();
     };
-    // pass 1: M = max over every contributor
-    for (int base = 0; base < ncc; base += 32) {
-        load_chunk(base);
-        if (tid < g) {
-            float mx = cs.M[tid];
-            for (int j = 0; j < 32; ++j) mx = fmaxf(mx, cs.m[tid][j]);
-            cs.M[tid] = mx;
+    // weighted sum of the batch; w of chunk position jc0 + jj
+    auto consume = [&](int jc0) {
+#pragma unroll
+        for (int k = 0; k < kOut4; ++k) {
+            const int i4 = tid + k * THREADS;
+            const int q = i4 < n4 ? (i4 * 4) / D : 0;
+#pragma unroll
+            for (int jj = 0; jj < kBatch; ++jj) {
+                const float w = (jc0 + jj < 32) ? cs.w[q][jc0 + jj] : 0.0f;
+                acc[k].x = fmaf(w, v[k][jj].x, acc[k].x);
+                acc[k].y = fmaf(w, v[k][jj].y, acc[k].y);
+                acc[k].z = fmaf(w, v[k][jj].z, acc[k].z);
+                acc[k].w = fmaf(w, v[k][jj].w, acc[k].w);
+            }
+        }
+    };
+    const int nj0 = ncc < 32 ? ncc : 32;
+    issue(0, nj0);                                   // in flight with the (m, l) loads below
+
+    // M per query (warp-uniform); the first chunk's (m, l) stay in registers
+    float Mq[kQW], m0[kQW], l0[kQW], Lq[kQW];
+#pragma unroll
+    for (int qi = 0; qi < kQW; ++qi) {
+        const int q = warp + qi * kWarps;
+        Mq[qi] = -INFINITY;
+        m0[qi] = -INFINITY;
+        l0[qi] = 0.0f;
+        Lq[qi] = 0.0f;
+        if (q < g) {
+            for (int base = 0; base < ncc; base += 32) {
+                const int j = base + lane;
+                float m = -INFINITY, l = 0.0f;
+                if (j < ncc) {
+                    const float* pp = part_of(j);
+                    m = __ldcg(pp + g * D + q);
+                    l = __ldcg(pp + g * D + g + q);
+                }
+                if (base == 0) {
+                    m0[qi] = m;
+                    l0[qi] = l;
+                }
+                Mq[qi] = fmaxf(Mq[qi], m);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) Mq[qi] = fmaxf(Mq[qi], __shfl_xor_sync(0xFFFFFFFFu, Mq[qi], o));
         }
     }
-    // pass 2: weights, L and the weighted sum of the O partials
+
     for (int base = 0; base < ncc; base += 32) {
-        if (ncc > 32) load_chunk(base);      // a single chunk is still in place
-        group_sync<THREADS, BAR>();
-        if (tid < g) {
-            const float M = cs.M[tid];
-            float lsum = cs.L[tid];
-            for (int j = 0; j < 32; ++j) {
-                const float mj = cs.m[tid][j];
-                const float w = (mj == -INFINITY) ? 0.0f : fast_exp2(mj - M);
-                lsum += w * cs.l[tid][j];
-                cs.l[tid][j] = w;                // l is replaced by the weight
-            }
-            cs.L[tid] = lsum;
-        }
-        group_sync<THREADS, BAR>();
         const int nj = ncc - base < 32 ? ncc - base : 32;
-        for (int j0 = 0; j0 < nj; j0 += kBatch) {
-            float4 v[kOut4][kBatch];
-            float w[kOut4][kBatch];
+        if (base > 0) group_sync<THREADS, BAR>();   // the previous chunk's weights are consumed
 #pragma unroll
-            for (int k = 0; k < kOut4; ++k) {          // every load of the batch in flight at once
-                const int i4 = tid + k * THREADS;
-                const int q = i4 < n4 ? (i4 * 4) / D : 0;
-#pragma unroll
-                for (int jj = 0; jj < kBatch; ++jj) {
-                    const int j = j0 + jj;
-                    const int sl = (j < nj && i4 < n4) ? cs.slot[j] : -1;
-                    w[k][jj] = sl >= 0 ? cs.l[q][j] : 0.0f;
-                    v[k][jj] = sl >= 0 ? __ldcg(reinterpret_cast<const float4*>(
-                                             p.partials + (int64_t)sl * slot_floats) + i4)
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int qi = 0; qi < kQW; ++qi) {
+            const int q = warp + qi * kWarps;
+            if (q < g) {
+                float m = m0[qi], l = l0[qi];
+                if (base > 0) {
+                    m = -INFINITY;
+                    l = 0.0f;
+                    if (lane < nj) {
+                        const float* pp = part_of(base + lane);
+                        m = __ldcg(pp + g * D + q);
+                        l = __ldcg(pp + g * D + g + q);
+                    }
                 }
+                const float w = (m == -INFINITY) ? 0.0f : fast_exp2(m - Mq[qi]);
+                float wl = w * l;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) wl += __shfl_xor_sync(0xFFFFFFFFu, wl, o);
+                Lq[qi] += wl;
+                cs.w[q][lane] = w;
             }
-#pragma unroll
-            for (int k = 0; k < kOut4; ++k)
-#pragma unroll
-                for (int jj = 0; jj < kBatch; ++jj) {
-                    acc[k].x = fmaf(w[k][jj], v[k][jj].x, acc[k].x);
-                    acc[k].y = fmaf(w[k][jj], v[k][jj].y, acc[k].y);
-                    acc[k].z = fmaf(w[k][jj], v[k][jj].z, acc[k].z);
-                    acc[k].w = fmaf(w[k][jj], v[k][jj].w, acc[k].w);
-                }
         }
+        group_sync<THREADS, BAR>();
+        for (int j0 = 0; j0 < nj; j0 += kBatch) {
+            if (base > 0 || j0 > 0) issue(base + j0, base + nj);
+            consume(j0);
+        }
+    }
+#pragma unroll
+    for (int qi = 0; qi < kQW; ++qi) {
+        const int q = warp + qi * kWarps;
+        if (q < g && lane == 0) cs.L[q] = Lq[qi];
     }
     group_sync<THREADS, BAR>();
 #pragma unroll

@@ -634,23 +634,14 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_attention_kern
             }
         }
         if (!whole) {
-            __threadfence();
             __syncthreads();
-            const int64_t c_first = cta_of(u.U0, T, N);
-            const int64_t c_last = cta_of(u.U1 - 1, T, N);
             if (tid == 0) {
-                // contributors: the CTAs with a non-empty range inside the unit's
-                // span (ranges are empty only when there are fewer tiles than CTAs)
-                int contributors = 0;
-                for (int64_t cc = c_first; cc <= c_last; ++cc)
-                    contributors += range_start(cc, T, N) < range_start(cc + 1, T, N);
-                const int prev = atomicAdd(&p.counters[(int64_t)u.b * p.Hkv + u.h], 1);
-                sm.last_flag = (prev == contributors - 1);
+                const int prev = arrive_split_unit(&p.counters[(int64_t)u.b * p.Hkv + u.h]);
+                sm.last_flag = (prev == unit_contributors(u.U0, u.U1, T, N) - 1);
             }
             __syncthreads();
             if (sm.last_flag) {
-                __threadfence();
-                combine_partials<D, NT, kWarps * 32>(p, sm.comb, u, T, N, c_first, c_last, slot_floats, tid, warp, lane);
+                combine_partials<D, NT, kWarps * 32>(p, sm.comb, u, T, N, slot_floats, tid, warp, lane);
                 if (tid == 0) atomicExch(&p.counters[(int64_t)u.b * p.Hkv + u.h], 0);
             }
         }

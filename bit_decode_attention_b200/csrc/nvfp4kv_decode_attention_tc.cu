@@ -101,8 +101,9 @@ struct __align__(1024) Smem {
     int32_t warp_tot[kThreads / 32];
     CombineSmem comb;
     uint32_t tmem_base;
-    int32_t last_flag;
+    int32_t n_sig;                                    // split units whose partial this CTA wrote
     int32_t n_pend;                                   // units this CTA must merge at its end
+    int64_t sig_gt[2];
     int64_t pend_gt[2];
     int32_t abort_flag;
 };
@@ -165,12 +166,6 @@ __device__ __forceinline__ bool softmax_any(bool v) {
     return r != 0;
 }
 
-__device__ __forceinline__ void tmem_ld_x4(uint32_t taddr, uint32_t* r) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(taddr)
-                 : "memory");
-}
 __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t* r) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
@@ -454,6 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
         mbar_init(&sm.mma_done, 1);
         fence_mbar_init();
         sm.abort_flag = 0;
+        sm.n_sig = 0;
         sm.n_pend = 0;
         // the first two tiles only: the CTA barrier below waits for this lane
         while (load_w < 2u && load_walk.next(sm.prefix, sm.lens, B, p.Hkv)) {
@@ -864,21 +860,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
                             part[g * 128 + g + q] = lt[q];
                         }
                 }
-                __threadfence();
-                softmax_sync();
-                const int64_t c_first = cta_of(u.U0, T, N);
-                const int64_t c_last = cta_of(u.U1 - 1, T, N);
-                if (t == 0) {
-                    int contributors = 0;
-                    for (int64_t cc = c_first; cc <= c_last; ++cc)
-                        contributors += range_start(cc, T, N) < range_start(cc + 1, T, N);
-                    const int prev = atomicAdd(&p.counters[(int64_t)u.b * p.Hkv + u.h], 1);
-                    sm.last_flag = (prev == contributors - 1);
-                }
-                softmax_sync();
-                // the merge waits until every role of this CTA is done and then
-                // runs on all its threads (a CTA is last for at most two units)
-                if (sm.last_flag && t == 0) sm.pend_gt[sm.n_pend++] = u.U0;
+                // arrival is counted after the roles finish, so that the
+                // fence and the atomic stay off this CTA's tile pipeline
+                if (t == 0) sm.sig_gt[sm.n_sig++] = u.U0;
             }
             softmax_sync();
             seg_lo = seg_hi;
@@ -891,14 +875,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
     tc::fence_after_sync();
     if (warp == kMmaWarp) tc::tmem_dealloc(tbase, C::kTmemCols);
 
-    // ---- split-K merges of the units this CTA finished last, on every thread ----
+    // ---- split-K: count this CTA's arrival at each split unit (one lane per
+    // unit, atomics in flight together); the last to arrive merges the unit
+    // on every thread ----
+    if (warp == 0) {
+        const int n_sig = sm.n_sig;
+        bool last = false;
+        int64_t gt = 0;
+        if (lane < n_sig) {
+            gt = sm.sig_gt[lane];
+            const Unit u = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, gt);
+            const int prev = arrive_split_unit(&p.counters[(int64_t)u.b * p.Hkv + u.h]);
+            last = prev == unit_contributors(u.U0, u.U1, T, N) - 1;
+        }
+        const uint32_t lm = __ballot_sync(0xFFFFFFFFu, last);
+        if (last) sm.pend_gt[__popc(lm & ((1u << lane) - 1u))] = gt;
+        if (lane == 0) sm.n_pend = __popc(lm);
+    }
+    __syncthreads();
     const int n_pend = sm.n_pend;
     for (int i = 0; i < n_pend; ++i) {
         const Unit u = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, sm.pend_gt[i]);
-        __threadfence();
-        combine_partials<128, NT, kThreads, 0>(p, sm.comb, u, T, N, cta_of(u.U0, T, N),
-                                               cta_of(u.U1 - 1, T, N), partial_slot_floats(p.g, 128),
-                                               tid, warp, lane);
+        combine_partials<128, NT, kThreads, 0>(p, sm.comb, u, T, N, partial_slot_floats(p.g, 128), tid,
+                                               warp, lane);
         if (tid == 0) atomicExch(&p.counters[(int64_t)u.b * p.Hkv + u.h], 0);
     }
 }

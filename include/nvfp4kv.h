@@ -179,7 +179,9 @@ size_t nvfp4_decode_attention_workspace(int B, int H_q, int H_kv, int D);
  *   workspace    device, >= nvfp4_decode_attention_workspace(...) bytes,
  *                zero-filled once (see above), 16-byte aligned
  * Lengths past S_max are clamped and reported as NVFP4_ERR_CAPACITY.
- * Batches larger than 512 sequences are processed in launches of 512. */
+ * Batches larger than 512 sequences are processed in launches of 512.
+ * NVFP4_ERR_UNSUPPORTED when min(B, 512) * H_kv * ceil(S_max / 32) exceeds
+ * 2^31 - 1 (the work split counts 32-token tiles in 32 bits). */
 nvfp4_status nvfp4_decode_attention(const void* q, nvfp4_dtype q_dtype, int H_q,
                                     const nvfp4_kv_plane* k, const nvfp4_kv_plane* v,
                                     const float* d_s_tensor_k, const float* d_s_tensor_v,

@@ -101,6 +101,11 @@ def test_argument_validation_without_gpu(lib):
     assert at(*args(3, k, v, dev, 1 << 30)) == INVALID            # H_q % H_kv
     assert at(*args(4, k, v_other, dev, 1 << 30)) == INVALID      # planes disagree
     assert at(*args(2 * 17, k, v, dev, 1 << 30)) == _native.NVFP4_ERR_UNSUPPORTED
+    # 2^10 KV heads x 2^21 tokens = 2^26 tiles of 32 tokens per sequence: fits
+    # 32-bit tile counts for one sequence, not for 2^6 of them
+    big1, big64 = _plane(B=1, H=1 << 10, S=1 << 21), _plane(B=64, H=1 << 10, S=1 << 21)
+    assert at(*args(1 << 10, big64, big64, dev, 1 << 30)) == _native.NVFP4_ERR_UNSUPPORTED
+    assert at(*args(1 << 10, big1, big1, dev, 16)) == WS           # passes the tile check
     assert at(dev, 0, 4, ctypes.byref(k), ctypes.byref(v), dev, dev, dev, ctypes.c_float(0.0),
               ctypes.c_void_p(68), dev, 1 << 30, None, None) == INVALID   # out misaligned
     assert at(*args(4, k, v, None, 0)) == WS
