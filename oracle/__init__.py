@@ -56,6 +56,20 @@ def lib():
                                                     ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                     i32p, ctypes.c_double, f64p]
         L.oracle_kv_bytes.argtypes = [ctypes.c_int64] * 5 + [ctypes.c_double]
+        L.oracle_nvfp4_reconstruct_planes.argtypes = [u8p, u8p, ctypes.c_int, ctypes.c_int,
+                                                      ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                                      i32p, f64p]
+        L.oracle_e8m0_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e8m0_value.restype = ctypes.c_double
+        L.oracle_mxfp4_quantize_block.argtypes = [f32p, u8p, u8p]
+        L.oracle_mxfp4_quantize_block.restype = ctypes.c_int
+        L.oracle_mxfp4_quantize_append.argtypes = [f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int, i32p, u8p, u8p, ctypes.c_int]
+        L.oracle_mxfp4_quantize_append.restype = ctypes.c_int
+        L.oracle_mxfp4_reconstruct_planes.argtypes = [u8p, u8p, ctypes.c_int, ctypes.c_int,
+                                                      ctypes.c_int, ctypes.c_int, i32p, f64p]
+        L.oracle_mxfp4_bits_per_element.argtypes = []
+        L.oracle_mxfp4_bits_per_element.restype = ctypes.c_double
         L.oracle_kv_bytes.restype = ctypes.c_double
         L.oracle_nvfp4_bits_per_element.argtypes = []
         L.oracle_nvfp4_bits_per_element.restype = ctypes.c_double
@@ -157,6 +171,70 @@ def dequant_planes(codes, scales, s_tensor, seq_lens):
                                 B, H_kv, S_max, D, np.float32(s_tensor),
                                 _p(seq_lens, ctypes.c_int32), _p(out, ctypes.c_uint8))
     return out
+
+
+def nvfp4_reconstruct_planes(codes, scales, s_tensor, seq_lens):
+    """fp64 x^ = value(code) * value(sb) * s_tensor, [B][H_kv][S_max][D] (unset slots 0)."""
+    B, H_kv, S_max, Dh = codes.shape
+    D = 2 * Dh
+    seq_lens = np.ascontiguousarray(seq_lens, np.int32)
+    out = np.zeros((B, H_kv, S_max, D), np.float64)
+    lib().oracle_nvfp4_reconstruct_planes(_p(np.ascontiguousarray(codes), ctypes.c_uint8),
+                                          _p(np.ascontiguousarray(scales), ctypes.c_uint8),
+                                          B, H_kv, S_max, D, np.float32(s_tensor),
+                                          _p(seq_lens, ctypes.c_int32), _p(out, ctypes.c_double))
+    return out
+
+
+# ---- MXFP4 ("MXFP4との比較": 32-element blocks, E8M0 scales) -------------------
+def e8m0_value(byte: int) -> float:
+    return lib().oracle_e8m0_value(byte)
+
+
+def mxfp4_quantize_block(x32):
+    """Return (status, packed 16 bytes, E8M0 scale byte) for 32 fp32 values."""
+    x32 = _f32(x32).ravel()
+    assert x32.size == 32
+    packed = np.zeros(16, np.uint8)
+    sb = np.zeros(1, np.uint8)
+    st = lib().oracle_mxfp4_quantize_block(_p(x32, ctypes.c_float), _p(packed, ctypes.c_uint8),
+                                           _p(sb, ctypes.c_uint8))
+    return int(st), packed, int(sb[0])
+
+
+def new_mxfp4_planes(B, H_kv, S_max, D):
+    codes = np.zeros((B, H_kv, S_max, D // 2), np.uint8)
+    scales = np.zeros((B, H_kv, S_max, D // 32), np.uint8)
+    return codes, scales
+
+
+def mxfp4_quantize_append(x_new, start, codes, scales):
+    """x_new fp32 [B][n_new][H_kv][D]; codes/scales are updated in place."""
+    x_new = _f32(x_new)
+    B, n_new, H_kv, D = x_new.shape
+    S_max = codes.shape[2]
+    start = np.ascontiguousarray(start, np.int32)
+    assert codes.flags.c_contiguous and scales.flags.c_contiguous
+    return int(lib().oracle_mxfp4_quantize_append(
+        _p(x_new, ctypes.c_float), B, n_new, H_kv, D, _p(start, ctypes.c_int32),
+        _p(codes, ctypes.c_uint8), _p(scales, ctypes.c_uint8), S_max))
+
+
+def mxfp4_reconstruct_planes(codes, scales, seq_lens):
+    """fp64 x^ = value(code) * 2^(e8m0 - 127), [B][H_kv][S_max][D] (unset slots 0)."""
+    B, H_kv, S_max, Dh = codes.shape
+    D = 2 * Dh
+    seq_lens = np.ascontiguousarray(seq_lens, np.int32)
+    out = np.zeros((B, H_kv, S_max, D), np.float64)
+    lib().oracle_mxfp4_reconstruct_planes(_p(np.ascontiguousarray(codes), ctypes.c_uint8),
+                                          _p(np.ascontiguousarray(scales), ctypes.c_uint8),
+                                          B, H_kv, S_max, D, _p(seq_lens, ctypes.c_int32),
+                                          _p(out, ctypes.c_double))
+    return out
+
+
+def mxfp4_bits_per_element() -> float:
+    return lib().oracle_mxfp4_bits_per_element()
 
 
 # ---- attention --------------------------------------------------------------

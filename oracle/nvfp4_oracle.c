@@ -224,6 +224,108 @@ void oracle_dequant_planes(const uint8_t* codes, const uint8_t* scales,
             }
 }
 
+/* The pages' reconstruction, x ~ x_q * s_block * s_tensor ([P3]
+ * "E2M1 + 2レベルスケーリング"), in fp64 without the FP8 rounding of R7. */
+void oracle_nvfp4_reconstruct_planes(const uint8_t* codes, const uint8_t* scales,
+                                     int B, int H_kv, int S_max, int D, float s_tensor,
+                                     const int32_t* seq_lens, double* out) {
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H_kv; ++h)
+            for (int t = 0; t < seq_lens[b]; ++t) {
+                int64_t slot = ((int64_t)b * H_kv + h) * S_max + t;
+                for (int d = 0; d < D; ++d) {
+                    uint8_t byte = codes[slot * (D / 2) + d / 2];
+                    uint8_t code = (d % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+                    uint8_t sb = scales[slot * (D / 16) + d / 16];
+                    out[slot * D + d] =
+                        oracle_e2m1_value(code) * oracle_e4m3_value(sb) * (double)s_tensor;
+                }
+            }
+}
+
+/* --------------------------------------------------------------------------
+ * MXFP4, the OCP format the pages compare NVFP4 with ([P3] "MXFP4との比較"):
+ * blocks of 32 elements, one E8M0 scale that can only be a power of two, no
+ * tensor scale.  E8M0 is a bare biased exponent: byte e + 127 is 2^e, 0xFF is
+ * NaN (R13).
+ * ------------------------------------------------------------------------ */
+double oracle_e8m0_value(uint8_t byte) {
+    if (byte == 0xFF) return NAN;
+    return ldexp(1.0, (int)byte - 127);
+}
+
+int oracle_mxfp4_quantize_block(const float* x32, uint8_t* packed16, uint8_t* scale_byte) {
+    double amax = 0.0;
+    for (int i = 0; i < 32; ++i) {
+        if (!isfinite(x32[i])) {                     /* R15 */
+            for (int j = 0; j < 16; ++j) packed16[j] = 0;
+            *scale_byte = 0xFF;
+            return ORACLE_ERR_NONFINITE;
+        }
+        double a = fabs((double)x32[i]);
+        if (a > amax) amax = a;
+    }
+    /* R13: X = 2^(floor(log2 amax) - 2), so amax / X lies in [4, 8): the
+     * block's largest element lands on the top binade of E2M1 (4 or 6). */
+    int e = -127;
+    if (amax > 0.0) {
+        int ex;
+        frexp(amax, &ex);                            /* amax = m 2^ex, 0.5 <= m < 1 */
+        e = (ex - 1) - 2;
+        if (e < -127) e = -127;
+        if (e > 127) e = 127;
+    }
+    double X = ldexp(1.0, e);
+    uint8_t codes[32];
+    for (int i = 0; i < 32; ++i)
+        codes[i] = oracle_e2m1_encode((float)((double)x32[i] / X));   /* R14 */
+    for (int j = 0; j < 16; ++j)                     /* R6 packing */
+        packed16[j] = (uint8_t)(codes[2 * j] | (codes[2 * j + 1] << 4));
+    *scale_byte = (uint8_t)(e + 127);
+    return ORACLE_OK;
+}
+
+int oracle_mxfp4_quantize_append(const float* x_new, int B, int n_new, int H_kv, int D,
+                                 const int32_t* start, uint8_t* codes, uint8_t* scales,
+                                 int S_max) {
+    if (D % 32 != 0 || B < 0 || n_new < 0 || H_kv <= 0) return ORACLE_ERR_ARG;
+    int status = ORACLE_OK;
+    for (int b = 0; b < B; ++b) {
+        if (start[b] < 0 || (int64_t)start[b] + n_new > S_max) {
+            status = ORACLE_ERR_CAPACITY;
+            continue;
+        }
+        for (int t = 0; t < n_new; ++t)
+            for (int h = 0; h < H_kv; ++h) {
+                const float* row = x_new + (((int64_t)b * n_new + t) * H_kv + h) * D;
+                int64_t slot = ((int64_t)b * H_kv + h) * S_max + (start[b] + t);
+                for (int blk = 0; blk < D / 32; ++blk) {
+                    int r = oracle_mxfp4_quantize_block(row + 32 * blk,
+                                                        codes + slot * (D / 2) + 16 * blk,
+                                                        scales + slot * (D / 32) + blk);
+                    if (r != ORACLE_OK && status == ORACLE_OK) status = r;
+                }
+            }
+    }
+    return status;
+}
+
+void oracle_mxfp4_reconstruct_planes(const uint8_t* codes, const uint8_t* scales,
+                                     int B, int H_kv, int S_max, int D,
+                                     const int32_t* seq_lens, double* out) {
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H_kv; ++h)
+            for (int t = 0; t < seq_lens[b]; ++t) {
+                int64_t slot = ((int64_t)b * H_kv + h) * S_max + t;
+                for (int d = 0; d < D; ++d) {
+                    uint8_t byte = codes[slot * (D / 2) + d / 2];
+                    uint8_t code = (d % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+                    uint8_t sb = scales[slot * (D / 32) + d / 32];
+                    out[slot * D + d] = oracle_e2m1_value(code) * oracle_e8m0_value(sb);
+                }
+            }
+}
+
 /* --------------------------------------------------------------------------
  * Decode attention.  [P3] "量子化・逆量子化フロー": FP8 attention and the
  * context matmul run on the dequantized cache; [P5] "Le type de Blackwell":
@@ -333,6 +435,9 @@ void oracle_decode_attention_nvfp4(const float* q,
  * the single fp32 tensor scale is negligible and left out.
  * ------------------------------------------------------------------------ */
 double oracle_nvfp4_bits_per_element(void) { return 4.0 + 8.0 / 16.0; }
+
+/* MXFP4 ([P3] "MXFP4との比較"): 4 code bits plus one 8-bit E8M0 scale per 32. */
+double oracle_mxfp4_bits_per_element(void) { return 4.0 + 8.0 / 32.0; }
 
 double oracle_kv_bytes(int64_t layers, int64_t n_h, int64_t d_h, int64_t s, int64_t b,
                        double bits_per_element) {

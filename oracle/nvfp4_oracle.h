@@ -12,7 +12,8 @@
  *        Sections used: "KV Cacheのメモリボトルネック" (memory formula),
  *        "E2M1 + 2レベルスケーリング" (format and two-level scaling),
  *        "量子化・逆量子化フロー" (quantize on append, dequantize to FP8,
- *        FP8 attention), "メモリ削減効果" (memory-reduction table).
+ *        FP8 attention), "メモリ削減効果" (memory-reduction table),
+ *        "MXFP4との比較" (MXFP4: 32-element blocks, E8M0 power-of-two scales).
  *   [P1] "TensorRT-LLM rc17 が SM121（DGX Spark）向けに NVFP4 MoE バックエンドと
  *        NVFP4 KV キャッシュを追加", section "物語の KV キャッシュ側"
  *        (values are dequantized from NVFP4 to FP8 before attention).
@@ -36,6 +37,15 @@
  *       code's sign bit copied to the FP8 sign bit (so -0 codes give 0x80).
  *   R8  Attention in fp64 over the FP8 values: query head h reads KV head
  *       h / (H_q/H_kv); empty sequences give a zero row.
+ *   R13 MXFP4 scale: the pages fix only "E8M0, powers of two".  The OCP MX
+ *       rule is taken: X = 2^e, e = floor(log2(amax_blk)) - 2 (2 is the
+ *       exponent of E2M1's largest value 6 = 1.5 * 2^2), clamped to
+ *       [-127, 127]; amax_blk == 0 gives e = -127.  E8M0 byte = e + 127.
+ *   R14 MXFP4 codes: code_i = E2M1(x_i / X) (exact, X is a power of two),
+ *       packed as R6; a block is 32 consecutive elements along head_dim of
+ *       one token; there is no tensor scale.
+ *   R15 A block holding NaN or +-Inf gets the E8M0 NaN byte 0xFF and zero
+ *       codes, and the append reports ORACLE_ERR_NONFINITE.
  */
 #ifndef NVFP4_ORACLE_H
 #define NVFP4_ORACLE_H
@@ -104,6 +114,30 @@ void    oracle_decode_attention_nvfp4(const float* q,
                                       int B, int H_q, int H_kv, int S_max, int D,
                                       const int32_t* seq_lens, double softmax_scale,
                                       double* out);
+
+/* ---- the exact reconstruction x^ = value(code) * value(sb) * s_tensor
+ * ([P3] "E2M1 + 2レベルスケーリング"), fp64 [B][H_kv][S_max][D], slots
+ * t < seq_lens[b] only.  Used to measure quantization error. */
+void    oracle_nvfp4_reconstruct_planes(const uint8_t* codes, const uint8_t* scales,
+                                        int B, int H_kv, int S_max, int D, float s_tensor,
+                                        const int32_t* seq_lens, double* out);
+
+/* ---- MXFP4 ([P3] "MXFP4との比較"; readings R13-R15) ----
+ * scales : uint8 [B][H_kv][S_max][D/32], one E8M0 byte per 32 elements;
+ * codes  : uint8 [B][H_kv][S_max][D/2] as for NVFP4. */
+double  oracle_e8m0_value(uint8_t byte);            /* 2^(byte - 127); NaN for 0xFF */
+/* Returns ORACLE_OK, or ORACLE_ERR_NONFINITE for a block with NaN/Inf (R15). */
+int     oracle_mxfp4_quantize_block(const float* x32, uint8_t* packed16, uint8_t* scale_byte);
+/* Same placement and capacity rules as oracle_quantize_append; returns
+ * ORACLE_ERR_CAPACITY or ORACLE_ERR_NONFINITE (capacity wins) or ORACLE_OK. */
+int     oracle_mxfp4_quantize_append(const float* x_new, int B, int n_new, int H_kv, int D,
+                                     const int32_t* start, uint8_t* codes, uint8_t* scales,
+                                     int S_max);
+/* x^ = value(code) * value(e8m0), fp64, slots t < seq_lens[b] only. */
+void    oracle_mxfp4_reconstruct_planes(const uint8_t* codes, const uint8_t* scales,
+                                        int B, int H_kv, int S_max, int D,
+                                        const int32_t* seq_lens, double* out);
+double  oracle_mxfp4_bits_per_element(void);
 
 /* ---- memory model ([P3] "KV Cacheのメモリボトルネック") ----
  * KV bytes = 2 (K and V) * layers * n_h * s * b * bytes per head vector. */

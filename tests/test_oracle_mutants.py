@@ -22,8 +22,8 @@ MUTANTS = [
      "float y = x16[i] / den;", "float y = x16[i] * den;",
      [pins.test_block_invariants]),
     ("nibble_order_swapped",
-     "(uint8_t)(codes[2 * j] | (codes[2 * j + 1] << 4))",
-     "(uint8_t)(codes[2 * j + 1] | (codes[2 * j] << 4))",
+     "packed8[j] = (uint8_t)(codes[2 * j] | (codes[2 * j + 1] << 4))",
+     "packed8[j] = (uint8_t)(codes[2 * j + 1] | (codes[2 * j] << 4))",
      [pins.check_all_quantize_golden]),
     ("e2m1_ties_to_odd",
      "(d == best_d && (c & 1) == 0)", "(d == best_d && (c & 1) == 1)",
@@ -64,6 +64,30 @@ MUTANTS = [
     ("kv_memory_without_scale_bits",
      "return 4.0 + 8.0 / 16.0;", "return 4.0;",
      [pins.test_memory_ratios_match_pages]),
+    ("mxfp4_exponent_off_by_one",
+     "e = (ex - 1) - 2;", "e = (ex - 1) - 1;",
+     [pins.check_all_mxfp4_golden, pins.test_mxfp4_block_invariants]),
+    ("mxfp4_no_low_clamp",
+     "if (e < -127) e = -127;", "if (e < -140) e = -140;",
+     [pins.check_all_mxfp4_golden]),
+    ("mxfp4_multiply_by_scale",
+     "codes[i] = oracle_e2m1_encode((float)((double)x32[i] / X));",
+     "codes[i] = oracle_e2m1_encode((float)((double)x32[i] * X));",
+     [pins.check_all_mxfp4_golden, pins.test_mxfp4_grid_round_trip]),
+    ("mxfp4_nibble_order_swapped",
+     "packed16[j] = (uint8_t)(codes[2 * j] | (codes[2 * j + 1] << 4));",
+     "packed16[j] = (uint8_t)(codes[2 * j + 1] | (codes[2 * j] << 4));",
+     [pins.check_all_mxfp4_golden]),
+    ("mxfp4_nonfinite_ignored",
+     "if (!isfinite(x32[i])) {", "if (0) {",
+     [pins.test_mxfp4_nonfinite_blocks]),
+    ("mxfp4_scale_bias_wrong",
+     "return ldexp(1.0, (int)byte - 127);", "return ldexp(1.0, (int)byte - 128);",
+     [pins.test_e8m0_values]),
+    ("nvfp4_reconstruction_without_tensor_scale",
+     "oracle_e2m1_value(code) * oracle_e4m3_value(sb) * (double)s_tensor;",
+     "oracle_e2m1_value(code) * oracle_e4m3_value(sb);",
+     [pins.test_nvfp4_reconstruction_matches_block_decode]),
 ]
 
 

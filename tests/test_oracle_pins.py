@@ -396,3 +396,171 @@ def test_memory_ratios_match_pages():
                       ("reduction_vs_fp16", 1 - nv / fp16), ("fraction_of_fp8", nv / fp8)]:
         want, tol = printed[name]
         assert abs(val - want) <= tol, (name, val, want)
+
+
+# --------------------------------------------------------------------------
+# MXFP4 ("MXFP4との比較": 32-element blocks, E8M0 power-of-two scales)
+# --------------------------------------------------------------------------
+def _golden_x32(xs):
+    x = np.zeros(32, np.float32)
+    vals = [float(t) for t in xs.split()]
+    x[:len(vals)] = np.array(vals, np.float32)
+    return x
+
+
+@pytest.mark.parametrize("row", read_golden("mxfp4_worked.txt"), ids=lambda r: r[0])
+def test_mxfp4_worked_examples(row):
+    name, xs, sb, packed = row
+    st, got_packed, got_sb = oracle.mxfp4_quantize_block(_golden_x32(xs))
+    assert st == 0
+    assert got_sb == int(sb, 16)
+    assert [int(b) for b in got_packed] == [int(t, 16) for t in packed.split()]
+
+
+def check_all_mxfp4_golden():
+    for row in read_golden("mxfp4_worked.txt"):
+        test_mxfp4_worked_examples(row)
+
+
+def test_e8m0_values():
+    # E8M0: a bare exponent with bias 127; 0xFF is NaN
+    assert oracle.e8m0_value(0x7F) == 1.0
+    assert oracle.e8m0_value(0x80) == 2.0
+    assert oracle.e8m0_value(0x7C) == 0.125
+    assert oracle.e8m0_value(0x00) == 2.0 ** -127
+    assert oracle.e8m0_value(0xFE) == 2.0 ** 127
+    assert np.isnan(oracle.e8m0_value(0xFF))
+
+
+def _mx_decode(packed, sb):
+    return np.array([oracle.e2m1_value(int(c)) for c in _unpack(packed)]) * oracle.e8m0_value(sb)
+
+
+def test_mxfp4_block_invariants():
+    rng = np.random.default_rng(11)
+    scale = np.exp(rng.normal(0, 6, (3000, 1)))
+    xs = (rng.standard_normal((3000, 32)) * scale).astype(np.float32)
+    for x in xs:
+        st, packed, sb = oracle.mxfp4_quantize_block(x)
+        assert st == 0
+        X = oracle.e8m0_value(sb)
+        amax = float(np.abs(x).max())
+        # the scale is the power of two that puts amax in [4, 8)
+        assert 4.0 <= amax / X < 8.0
+        codes = _unpack(packed)
+        deq = _mx_decode(packed, sb)
+        err = np.abs(x.astype(np.float64) - deq)
+        # the largest element takes code 4 or 6 ...
+        imax = int(np.argmax(np.abs(x)))
+        assert abs(oracle.e2m1_value(int(codes[imax]))) in (4.0, 6.0)
+        # ... every element is within half a grid step (2X at the top, where
+        # values past 6X saturate) and within X/4 below 2X
+        assert np.all(err <= 2.0 * X)
+        small = np.abs(x) < 2.0 * X
+        assert np.all(err[small] <= 0.25 * X)
+        # negating x flips the code signs only
+        _, packed_n, sb_n = oracle.mxfp4_quantize_block(-x)
+        assert sb_n == sb
+        np.testing.assert_array_equal(_unpack(packed_n), codes ^ 0x8)
+
+
+def test_mxfp4_grid_round_trip():
+    # data already on the MXFP4 grid (top element +-4 or +-6) comes back exactly
+    rng = np.random.default_rng(5)
+    for _ in range(500):
+        e = int(rng.integers(-120, 120))
+        codes = rng.integers(0, 16, 32).astype(np.uint8)
+        codes[int(rng.integers(32))] = (0x6 if rng.random() < 0.5 else 0x7) | (0x8 if rng.random() < 0.5 else 0)
+        x = (np.array([oracle.e2m1_value(int(c)) for c in codes]) * 2.0 ** e).astype(np.float32)
+        st, packed, sb = oracle.mxfp4_quantize_block(x)
+        assert st == 0 and sb == e + 127
+        got = _unpack(packed)
+        np.testing.assert_array_equal(got & 0x7, codes & 0x7)
+        nz = (codes & 0x7) != 0
+        np.testing.assert_array_equal(got[nz], codes[nz])
+
+
+def test_mxfp4_nonfinite_blocks():
+    for bad in (np.nan, np.inf, -np.inf):
+        x = np.ones(32, np.float32)
+        x[17] = bad
+        st, packed, sb = oracle.mxfp4_quantize_block(x)
+        assert st == 4 and sb == 0xFF and not packed.any()
+    B, H, S, D = 2, 1, 16, 64
+    codes, scales = oracle.new_mxfp4_planes(B, H, S, D)
+    x = np.ones((B, 1, H, D), np.float32)
+    x[1, 0, 0, 40] = np.nan                    # second block of sequence 1
+    assert oracle.mxfp4_quantize_append(x, [0, 0], codes, scales) == 4
+    assert scales[1, 0, 0, 1] == 0xFF and scales[1, 0, 0, 0] == 0x7D   # amax 1 -> e -2
+    assert scales[0, 0, 0, 1] != 0xFF
+    # a capacity failure is reported ahead of a non-finite block
+    assert oracle.mxfp4_quantize_append(x, [0, S], codes, scales) == 3
+
+
+def test_mxfp4_append_placement_and_capacity():
+    rng = np.random.default_rng(9)
+    B, n_new, H, S, D = 3, 5, 2, 32, 128
+    x = rng.standard_normal((B, n_new, H, D)).astype(np.float32)
+    start = np.array([0, 7, 28], np.int32)               # the last one does not fit
+    codes, scales = oracle.new_mxfp4_planes(B, H, S, D)
+    assert oracle.mxfp4_quantize_append(x, start, codes, scales) == 3
+    for b in range(B):
+        for t in range(n_new):
+            for h in range(H):
+                slot = start[b] + t
+                for blk in range(D // 32):
+                    if b == 2:
+                        assert slot >= S or not codes[b, h, slot].any()
+                        continue
+                    _, pk, sb = oracle.mxfp4_quantize_block(x[b, t, h, 32 * blk:32 * blk + 32])
+                    np.testing.assert_array_equal(codes[b, h, slot, 16 * blk:16 * blk + 16], pk)
+                    assert scales[b, h, slot, blk] == sb
+    assert not codes[2].any() and not scales[2].any()
+
+
+def test_mxfp4_bits_per_element():
+    # 4 code bits plus an 8-bit scale per 32 elements; NVFP4 pays one per 16
+    assert oracle.mxfp4_bits_per_element() == 4.25
+    assert oracle.nvfp4_bits_per_element() - oracle.mxfp4_bits_per_element() == 0.25
+
+
+def test_nvfp4_reconstruction_matches_block_decode():
+    rng = np.random.default_rng(2)
+    B, H, S, D = 1, 2, 16, 64
+    x = (rng.standard_normal((B, 3, H, D)) * 3).astype(np.float32)
+    st = np.float32(0.02)
+    codes, scales = oracle.new_planes(B, H, S, D)
+    oracle.quantize_append(x, [4], st, codes, scales)
+    rec = oracle.nvfp4_reconstruct_planes(codes, scales, st, [7])
+    for t in range(3):
+        for h in range(H):
+            for blk in range(D // 16):
+                pk, sb = oracle.quantize_block(x[0, t, h, 16 * blk:16 * blk + 16], st)
+                want = np.array([oracle.e2m1_value(int(c)) for c in _unpack(pk)]) \
+                    * oracle.e4m3_value(sb) * float(st)
+                np.testing.assert_array_equal(rec[0, h, 4 + t, 16 * blk:16 * blk + 16], want)
+    assert not rec[0, :, :4].any() and not rec[0, :, 7:].any()
+
+
+def test_mse_ordering_nvfp4_below_mxfp4():
+    """The pages' comparison table gives NVFP4 a smaller quantization error
+    than MXFP4 (MSE 0.08 against 0.72 on data they do not describe, so only the
+    ordering is checked), which they attribute to the E4M3 block scale.  On the
+    long-context K/V recipe (N(0,1) x per-channel log-normal(0,1), 0.1 % of the
+    elements N(0,30) outliers) both codecs quantize the same tokens."""
+    rng = np.random.default_rng(21)
+    B, n, H, D = 1, 256, 4, 128
+    chan = np.exp(rng.normal(0, 1, (1, 1, H, D)))
+    x = rng.standard_normal((B, n, H, D)) * chan
+    out = rng.random(x.shape) < 1e-3
+    x[out] = rng.normal(0, 30, out.sum())
+    x = x.astype(np.float32)
+    st = oracle.tensor_scale(x)[1]
+    c16, s16 = oracle.new_planes(B, H, n, D)
+    oracle.quantize_append(x, [0], st, c16, s16)
+    c32, s32 = oracle.new_mxfp4_planes(B, H, n, D)
+    assert oracle.mxfp4_quantize_append(x, [0], c32, s32) == 0
+    ref = x.transpose(0, 2, 1, 3).astype(np.float64)          # [B][H][n][D], the planes' order
+    mse_nv = np.mean((oracle.nvfp4_reconstruct_planes(c16, s16, st, [n]) - ref) ** 2)
+    mse_mx = np.mean((oracle.mxfp4_reconstruct_planes(c32, s32, [n]) - ref) ** 2)
+    assert mse_nv < mse_mx
