@@ -220,6 +220,20 @@ class DecodeWorkload:
             self.out.append(torch.empty(B, Hq, D, dtype=torch.float32, device=dev))
         elems = 2 * B * L0 * Hkv * D
         self.prefill_bytes = replicas * (elems * self.xk_d.element_size() + elems * 9 // 16)
+        # the MXFP4 comparison codec on the same prefill (32-element blocks, E8M0
+        # scales): 0.53125 B written per element; timed, then freed
+        mk = nv.KVPlane.allocate_mxfp4(B, Hkv, self.S_max, D)
+        mv = nv.KVPlane.allocate_mxfp4(B, Hkv, self.S_max, D)
+        reps = 3
+        ev[0].record()
+        for _ in range(reps):
+            nv.mxfp4_kv_quantize_append(self.xk_d, zeros, mk, status=self.status)
+            nv.mxfp4_kv_quantize_append(self.xv_d, zeros, mv, status=self.status)
+        ev[1].record()
+        torch.cuda.synchronize()
+        self.mx_prefill_ms = ev[0].elapsed_time(ev[1]) / reps
+        self.mx_prefill_bytes = elems * self.xk_d.element_size() + elems * 17 // 32
+        del mk, mv
         self.start = torch.full((B,), L0, dtype=torch.int32, device=dev)
         self.lens = torch.full((B,), L0 + 1 if with_append else L0, dtype=torch.int32, device=dev)
         self.ws = nv.new_workspace(B, Hq, Hkv, D)
@@ -553,7 +567,8 @@ def main():
         "device_status": status,
     }
     aux = {"calib_gbs": wl.calib_bytes / (wl.calib_ms / 1e3) / 1e9,
-           "prefill_quantize_gbs": wl.prefill_bytes / (wl.prefill_ms / 1e3) / 1e9}
+           "prefill_quantize_gbs": wl.prefill_bytes / (wl.prefill_ms / 1e3) / 1e9,
+           "mxfp4_prefill_quantize_gbs": wl.mx_prefill_bytes / (wl.mx_prefill_ms / 1e3) / 1e9}
     del wl
     torch.cuda.empty_cache()
     if not args.no_aux:

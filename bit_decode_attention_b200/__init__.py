@@ -27,6 +27,7 @@ __all__ = [
     "nvfp4_kv_quantize_append_kv",
     "nvfp4_kv_dequant_fp8", "nvfp4_decode_attention_workspace", "nvfp4_decode_attention",
     "nvfp4_version", "NativeError", "nvfp4_decode_attention_noalloc",
+    "mxfp4_cache_bytes", "mxfp4_kv_quantize_append",
 ]
 
 
@@ -67,6 +68,13 @@ class KVPlane:
     def allocate(cls, B: int, H_kv: int, S_max: int, D: int, device="cuda") -> "KVPlane":
         codes = torch.zeros(B, H_kv, S_max, D // 2, dtype=torch.uint8, device=device)
         scales = torch.zeros(B, H_kv, S_max, D // 16, dtype=torch.uint8, device=device)
+        return cls(codes, scales)
+
+    @classmethod
+    def allocate_mxfp4(cls, B: int, H_kv: int, S_max: int, D: int, device="cuda") -> "KVPlane":
+        """An MXFP4 plane: the same codes, scales uint8 [B][H_kv][S_max][D/32] (E8M0)."""
+        codes = torch.zeros(B, H_kv, S_max, D // 2, dtype=torch.uint8, device=device)
+        scales = torch.zeros(B, H_kv, S_max, D // 32, dtype=torch.uint8, device=device)
         return cls(codes, scales)
 
     @property
@@ -127,6 +135,26 @@ def nvfp4_kv_quantize_append_kv(x_k: torch.Tensor, x_v: torch.Tensor, start_pos:
                                                    _ptr(s_tensor_v), ctypes.byref(pk), ctypes.byref(pv),
                                                    _ptr(status), _stream(stream))
     _native.check("nvfp4_kv_quantize_append_kv", st)
+
+
+def mxfp4_cache_bytes(B: int, H_kv: int, S_max: int, D: int) -> int:
+    return int(_native.lib().mxfp4_cache_bytes(B, H_kv, S_max, D))
+
+
+def mxfp4_kv_quantize_append(x_new: torch.Tensor, start_pos: torch.Tensor, plane: KVPlane,
+                             new_lens: Optional[torch.Tensor] = None,
+                             status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Quantize x_new [B][n_new][H_kv][D] to MXFP4 (32-element blocks, E8M0
+    scales) and write it at slots start_pos[b]... of an MXFP4 `plane`."""
+    _need_cuda(x_new, start_pos, new_lens, status)
+    B, H, S, D = plane.shape
+    if plane.scales.shape[-1] != D // 32:
+        raise ValueError("an MXFP4 plane holds D/32 scale bytes per token (KVPlane.allocate_mxfp4)")
+    pl = plane.struct()
+    st = _native.lib().mxfp4_kv_quantize_append(_ptr(x_new), _dtype_code(x_new), x_new.shape[1],
+                                                _ptr(start_pos), _ptr(new_lens), ctypes.byref(pl),
+                                                _ptr(status), _stream(stream))
+    _native.check("mxfp4_kv_quantize_append", st)
 
 
 def nvfp4_kv_dequant_fp8(plane: KVPlane, s_tensor: torch.Tensor, seq_lens: torch.Tensor,

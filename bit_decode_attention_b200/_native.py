@@ -34,6 +34,8 @@ EXPORTS = (
     "nvfp4_decode_attention_workspace",
     "nvfp4_decode_attention",
     "nvfp4_decode_attention_noalloc",
+    "mxfp4_cache_bytes",
+    "mxfp4_kv_quantize_append",
 )
 
 
@@ -91,6 +93,10 @@ def lib():
     L.nvfp4_decode_attention_noalloc.argtypes = [vp, i32, i32, plane_p, plane_p, vp, vp, vp, f32, vp,
                                                  vp, vp]
     L.nvfp4_decode_attention_noalloc.restype = i32
+    L.mxfp4_cache_bytes.argtypes = [i32, i32, i32, i32]
+    L.mxfp4_cache_bytes.restype = sz
+    L.mxfp4_kv_quantize_append.argtypes = [vp, i32, i32, vp, vp, plane_p, vp, vp]
+    L.mxfp4_kv_quantize_append.restype = i32
     _lib = L
     return L
 

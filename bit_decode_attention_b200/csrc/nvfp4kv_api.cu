@@ -124,6 +124,25 @@ nvfp4_status nvfp4_kv_quantize_append_kv(const void* x_k, const void* x_v, nvfp4
                                                d_status, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t mxfp4_cache_bytes(int B, int H_kv, int S_max, int D) {
+    if (B < 0 || H_kv <= 0 || S_max < 0 || D <= 0 || (D % 32) != 0) return 0;
+    return (size_t)B * H_kv * S_max * (size_t)(D / 2 + D / 32);
+}
+
+nvfp4_status mxfp4_kv_quantize_append(const void* x_new, nvfp4_dtype dtype, int n_new,
+                                      const int32_t* d_start_pos, int32_t* d_new_lens,
+                                      const nvfp4_kv_plane* plane, int32_t* d_status,
+                                      nvfp4_stream_t stream) {
+    if (!plane_ok(plane) || n_new < 0 || d_start_pos == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (dtype != NVFP4_IN_BF16 && dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
+    if (d_new_lens != nullptr && d_new_lens == d_start_pos) return NVFP4_ERR_INVALID_ARG;
+    if (n_new == 0 || plane->B == 0) return NVFP4_OK;
+    if (x_new == nullptr || !aligned16(x_new)) return NVFP4_ERR_INVALID_ARG;
+    return from_cuda(launch_mxfp4_quantize_append(x_new, dtype == NVFP4_IN_F32, n_new, d_start_pos,
+                                                  d_new_lens, *plane, d_status,
+                                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
 nvfp4_status nvfp4_kv_dequant_fp8(const nvfp4_kv_plane* plane, const float* d_s_tensor,
                                   const int32_t* d_seq_lens, uint8_t* out_e4m3, int32_t* d_status,
                                   nvfp4_stream_t stream) {

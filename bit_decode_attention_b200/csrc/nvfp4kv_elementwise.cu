@@ -250,6 +250,101 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(
     }
 }
 
+// ---------------------------------------------------------------------------
+// MXFP4 quantize + append: the OCP MX format the NVFP4 page compares with
+// ("MXFP4との比較": 32-element blocks, one E8M0 power-of-two scale each, no
+// tensor scale).  One thread per block.
+// The OCP exponent is floor(log2 amax) - 2, clamped to -127, and the E8M0 byte
+// adds the bias 127.  For amax with fp32 exponent field E that is
+// max(E - 129, -127) + 127 = max(E - 2, 0), subnormal and zero amax (E = 0)
+// included.  Scaling by 2^(127 - byte) is then exact and leaves every element
+// below 8 in magnitude; values past 6 saturate in the E2M1 conversion.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t mxfp4_quantize_block(const float (&a)[16], const float (&b)[16],
+                                                         uint4& packed, bool& nonfinite) {
+    float amax = 0.0f;
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float x = fabsf(a[i]), y = fabsf(b[i]);
+        bad |= !(x <= 3.4028234663852886e38f) || !(y <= 3.4028234663852886e38f);   // NaN or Inf
+        amax = fmaxf(amax, fmaxf(x, y));
+    }
+    nonfinite = bad;
+    if (bad) {                                       // E8M0 NaN scale, zero codes
+        packed = make_uint4(0u, 0u, 0u, 0u);
+        return 0xFFu;
+    }
+    const uint32_t E = __float_as_uint(amax) >> 23;
+    const uint32_t sb = E >= 2u ? E - 2u : 0u;
+    const float inv = __uint_as_float((254u - sb) << 23);   // 2^(127 - sb), a normal float
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        w[i / 8] |= e2m1_from_float(__fmul_rn(a[i], inv)) << (4 * (i % 8));
+        w[2 + i / 8] |= e2m1_from_float(__fmul_rn(b[i], inv)) << (4 * (i % 8));
+    }
+    packed = make_uint4(w[0], w[1], w[2], w[3]);
+    return sb;
+}
+
+template <bool F32>
+__global__ void __launch_bounds__(256) mxfp4_quantize_append_kernel(
+    const void* __restrict__ x_new, int B, int n_new, int Hkv, int D,
+    const int32_t* __restrict__ start_pos, int32_t* __restrict__ new_lens, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales, int S_max, int32_t* __restrict__ status) {
+    const int nblk = D / 32;
+    const int64_t total = (int64_t)B * Hkv * n_new * nblk;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int blk = (int)(i % nblk);
+        int64_t r = i / nblk;
+        const int t = (int)(r % n_new);
+        r /= n_new;
+        const int h = (int)(r % Hkv);
+        const int b = (int)(r / Hkv);
+        const bool leader = (t == 0 && h == 0 && blk == 0);
+        const int start = start_pos[b];
+        if (start < 0 || (int64_t)start + n_new > S_max) {
+            if (leader) report(status, NVFP4_ERR_CAPACITY);
+            continue;
+        }
+        if (leader && new_lens != nullptr) new_lens[b] = start + n_new;
+        const int64_t elem = (((int64_t)b * n_new + t) * Hkv + h) * D + 32 * blk;
+        float va[16], vb[16];
+        load16<F32>(x_new, elem, va);
+        load16<F32>(x_new, elem + 16, vb);
+        uint4 packed;
+        bool bad;
+        const uint32_t sb = mxfp4_quantize_block(va, vb, packed, bad);
+        if (bad) report(status, NVFP4_ERR_NONFINITE);
+        const int64_t slot = ((int64_t)b * Hkv + h) * S_max + start + t;
+        *reinterpret_cast<uint4*>(codes + slot * (D / 2) + 16 * blk) = packed;
+        scales[slot * (D / 32) + blk] = (uint8_t)sb;
+    }
+}
+
+cudaError_t launch_mxfp4_quantize_append(const void* x_new, bool f32, int n_new,
+                                         const int32_t* d_start_pos, int32_t* d_new_lens,
+                                         const nvfp4_kv_plane& pl, int32_t* d_status,
+                                         cudaStream_t stream) {
+    const int64_t total = (int64_t)pl.B * pl.H_kv * n_new * (pl.D / 32);
+    if (total == 0) return cudaSuccess;
+    const int threads = 256;
+    int64_t grid = (total + threads - 1) / threads;
+    const int64_t cap = 16L * device_sm_count();
+    if (grid > cap) grid = cap;
+    if (f32)
+        mxfp4_quantize_append_kernel<true><<<(int)grid, threads, 0, stream>>>(
+            x_new, pl.B, n_new, pl.H_kv, pl.D, d_start_pos, d_new_lens, pl.codes, pl.scales, pl.S_max,
+            d_status);
+    else
+        mxfp4_quantize_append_kernel<false><<<(int)grid, threads, 0, stream>>>(
+            x_new, pl.B, n_new, pl.H_kv, pl.D, d_start_pos, d_new_lens, pl.codes, pl.scales, pl.S_max,
+            d_status);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_quantize_append_kv(const void* x_k, const void* x_v, bool f32, int n_new,
                                       const int32_t* d_start_pos, int32_t* d_new_lens,
                                       const float* d_st_k, const float* d_st_v,

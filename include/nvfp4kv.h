@@ -136,6 +136,31 @@ nvfp4_status nvfp4_kv_quantize_append(const void* x_new, nvfp4_dtype dtype, int 
                                       const float* d_s_tensor, const nvfp4_kv_plane* plane,
                                       int32_t* d_status, nvfp4_stream_t stream);
 
+/* MXFP4 cache plane bytes: B * H_kv * S_max * (D/2 + D/32) -- 4 code bits
+ * plus one E8M0 scale byte per 32 elements = 4.25 bits per element.  Returns
+ * 0 for invalid sizes (D must be a multiple of 32). */
+size_t mxfp4_cache_bytes(int B, int H_kv, int S_max, int D);
+
+/* Quantize n_new tokens per sequence to MXFP4 and append them to a plane:
+ * the OCP format that [NVFP4-KV] "MXFP4との比較" compares NVFP4 with --
+ * 32-element blocks along head_dim, one E8M0 (power-of-two) scale per block,
+ * no tensor scale.  The scale exponent is floor(log2(amax_blk)) - 2 clamped
+ * to [-127, 127] (the OCP MX rule; the page fixes only block size and scale
+ * type), stored as the E8M0 byte exponent + 127; codes are
+ * E2M1_RNE_sat(x / 2^exponent), packed as for NVFP4.
+ *   x_new, dtype, n_new, d_start_pos, d_new_lens, d_status, stream: as for
+ *                nvfp4_kv_quantize_append
+ *   plane        codes [B][H_kv][S_max][D/2] and scales [B][H_kv][S_max][D/32]
+ *                (one E8M0 byte per 32 elements), both 16-byte aligned
+ * A sequence with start < 0 or start + n_new > S_max is skipped and
+ * NVFP4_ERR_CAPACITY goes to *d_status; a block holding NaN or Inf gets the
+ * E8M0 NaN byte 0xFF and zero codes, and NVFP4_ERR_NONFINITE goes to
+ * *d_status (the first error reported wins).  n_new == 0 is a no-op. */
+nvfp4_status mxfp4_kv_quantize_append(const void* x_new, nvfp4_dtype dtype, int n_new,
+                                      const int32_t* d_start_pos, int32_t* d_new_lens,
+                                      const nvfp4_kv_plane* plane, int32_t* d_status,
+                                      nvfp4_stream_t stream);
+
 /* Quantize-append the same new tokens into the K and the V plane in one
  * launch ([NVFP4-KV] "量子化・逆量子化フロー": K and V are both quantized
  * on append).  Same results, arguments and errors as two calls of

@@ -27,7 +27,7 @@ def declared_functions():
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
         text = open(h).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-        names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(nvfp4_\w+)\s*\(", text, flags=re.M)
+        names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b((?:nvfp4|mxfp4)_\w+)\s*\(", text, flags=re.M)
     return sorted(set(names))
 
 
@@ -55,6 +55,12 @@ def test_cache_bytes_matches_oracle_memory_model(lib):
         assert 2 * plane == oracle.kv_bytes(1, H, D, S, B, oracle.nvfp4_bits_per_element())
     assert lib.nvfp4_cache_bytes(1, 0, 16, 128) == 0
     assert lib.nvfp4_cache_bytes(1, 1, 16, 40) == 0
+    # MXFP4: 4.25 bits per element (one E8M0 byte per 32 elements)
+    for B, H, S, D in [(8, 8, 4096, 128), (3, 2, 48, 64)]:
+        plane = lib.mxfp4_cache_bytes(B, H, S, D)
+        assert plane == B * H * S * (D // 2 + D // 32)
+        assert 2 * plane == oracle.kv_bytes(1, H, D, S, B, oracle.mxfp4_bits_per_element())
+    assert lib.mxfp4_cache_bytes(1, 1, 16, 48) == 0
 
 
 def test_workspace_size(lib):
@@ -110,6 +116,14 @@ def test_argument_validation_without_gpu(lib):
               ctypes.c_void_p(68), dev, 1 << 30, None, None) == INVALID   # out misaligned
     assert at(*args(4, k, v, None, 0)) == WS
     assert at(*args(4, k, v, dev, 16)) == WS
+    mx = lib.mxfp4_kv_quantize_append
+    mxp = _plane(D=128, scales=32)
+    assert mx(dev, 0, 1, dev, None, ctypes.byref(bad_s), None, None) == INVALID
+    assert mx(dev, 7, 1, dev, None, ctypes.byref(mxp), None, None) == INVALID       # dtype
+    assert mx(dev, 0, 1, dev, dev, ctypes.byref(mxp), None, None) == INVALID        # aliasing
+    assert mx(ctypes.c_void_p(72), 0, 1, dev, None, ctypes.byref(mxp), None, None) == INVALID
+    assert mx(dev, 0, 1, None, None, ctypes.byref(mxp), None, None) == INVALID      # no start
+    assert mx(dev, 0, 0, dev, None, ctypes.byref(mxp), None, None) == 0             # no-op
     cal = lib.nvfp4_calib_tensor_scale
     assert cal(dev, 0, -1, dev, None, None) == INVALID
     assert cal(dev, 0, 10, None, None, None) == INVALID

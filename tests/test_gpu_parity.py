@@ -276,3 +276,102 @@ def test_quantize_append_kv_matches_two_calls(nv, dtype):
         assert oracle.quantize_append(x[1:2].numpy(), np.array([5], np.int32), st_o, oc, os_) == 0
         np.testing.assert_array_equal(pl.codes[1].cpu().numpy(), oc[0])
         np.testing.assert_array_equal(pl.scales[1].cpu().numpy(), os_[0])
+
+
+# ---------------------------------------------------------------------------
+# MXFP4 codec: the OCP format the pages compare NVFP4 with
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_mxfp4_quantize_append_bit_exact(nv, dtype, D):
+    w = synthetic.shrink(synthetic.get("long64k"), B=3, Hq=8, Hkv=2, D=D, dtype=dtype)
+    n_new = 37
+    x = synthetic.kv_tokens(w, n_new, "k")
+    start = np.array([0, 5, 100], np.int32)
+    S_max = synthetic.capacity(100 + n_new)
+    plane = nv.KVPlane.allocate_mxfp4(w.B, w.Hkv, S_max, D)
+    lens = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.mxfp4_kv_quantize_append(to_dev(x, dtype), torch.from_numpy(start).cuda(), plane, new_lens=lens,
+                                status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert lens.tolist() == (start + n_new).tolist()
+    oc, os_ = oracle.new_mxfp4_planes(w.B, w.Hkv, S_max, D)
+    assert oracle.mxfp4_quantize_append(x.numpy(), start, oc, os_) == 0
+    np.testing.assert_array_equal(plane.codes.cpu().numpy(), oc)
+    np.testing.assert_array_equal(plane.scales.cpu().numpy(), os_)
+
+
+def test_mxfp4_special_blocks_bit_exact(nv):
+    rows = synthetic.special_blocks(128)
+    extra = torch.zeros(4, 128)
+    extra[0, :3] = torch.tensor([3e38, -1.0, 1e-30])           # top of the exponent range
+    extra[1, :2] = torch.tensor([7.346839692639297e-40, -3.6734198463196485e-40])   # subnormal amax
+    extra[2, ::5] = 6.0 * 2.0 ** -100                         # exact grid values, low exponent
+    extra[3, :] = torch.linspace(-8.0, 8.0, 128)              # every E2M1 tie within one block
+    for dtype in ("f32", "bf16"):
+        src = torch.cat([rows, extra]) if dtype == "f32" else rows
+        x = src.to(torch.bfloat16).float() if dtype == "bf16" else src
+        n = x.shape[0]
+        x = x.view(1, n, 1, 128).contiguous()
+        plane = nv.KVPlane.allocate_mxfp4(1, 1, 16, 128)
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        nv.mxfp4_kv_quantize_append(to_dev(x, dtype), torch.zeros(1, dtype=torch.int32, device="cuda"),
+                                    plane, status=status)
+        torch.cuda.synchronize()
+        assert status.item() == 0
+        oc, os_ = oracle.new_mxfp4_planes(1, 1, 16, 128)
+        assert oracle.mxfp4_quantize_append(x.numpy(), np.zeros(1, np.int32), oc, os_) == 0
+        np.testing.assert_array_equal(plane.codes[0, 0, :n].cpu().numpy(), oc[0, 0, :n])
+        np.testing.assert_array_equal(plane.scales[0, 0, :n].cpu().numpy(), os_[0, 0, :n])
+
+
+def test_mxfp4_nonfinite_blocks_and_capacity(nv):
+    B, H, S, D = 3, 2, 16, 64
+    x = torch.ones(B, 2, H, D)
+    x[0, 1, 1, 40] = float("nan")
+    x[1, 0, 0, 3] = float("inf")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    plane = nv.KVPlane.allocate_mxfp4(B, H, S, D)
+    start = np.array([0, 3, 6], np.int32)
+    nv.mxfp4_kv_quantize_append(x.cuda(), torch.from_numpy(start).cuda(), plane, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == nv.NVFP4_ERR_NONFINITE
+    oc, os_ = oracle.new_mxfp4_planes(B, H, S, D)
+    assert oracle.mxfp4_quantize_append(x.numpy(), start, oc, os_) == 4
+    np.testing.assert_array_equal(plane.codes.cpu().numpy(), oc)
+    np.testing.assert_array_equal(plane.scales.cpu().numpy(), os_)
+    assert os_[0, 1, 1, 1] == 0xFF and os_[1, 0, 3, 0] == 0xFF
+    # a sequence past its capacity is skipped and reported; new_lens only for the others
+    status.zero_()
+    lens = torch.full((B,), -7, dtype=torch.int32, device="cuda")
+    start = np.array([0, 15, 14], np.int32)
+    plane2 = nv.KVPlane.allocate_mxfp4(B, H, S, D)
+    y = torch.ones(B, 2, H, D)
+    nv.mxfp4_kv_quantize_append(y.cuda(), torch.from_numpy(start).cuda(), plane2, new_lens=lens,
+                                status=status)
+    torch.cuda.synchronize()
+    assert status.item() == nv.NVFP4_ERR_CAPACITY
+    assert lens.tolist() == [2, -7, 16]
+    assert not plane2.codes[1].any().item() and not plane2.scales[1].any().item()
+
+
+def test_mxfp4_error_above_nvfp4_on_device_codes(nv):
+    # the pages' ordering (NVFP4 < MXFP4 quantization error) on the planes the
+    # device wrote for the long-context K recipe
+    w = synthetic.shrink(synthetic.get("long64k"), B=1, Hq=8, Hkv=2)
+    n = 512
+    x = synthetic.kv_tokens(w, n, "k")
+    xd = to_dev(x, "bf16")
+    start = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = nv.nvfp4_calib_tensor_scale(xd)
+    p16 = nv.KVPlane.allocate(1, w.Hkv, n, 128)
+    p32 = nv.KVPlane.allocate_mxfp4(1, w.Hkv, n, 128)
+    nv.nvfp4_kv_quantize_append(xd, start, st, p16)
+    nv.mxfp4_kv_quantize_append(xd, start, p32)
+    ref = x.numpy().transpose(0, 2, 1, 3).astype(np.float64)
+    rec16 = oracle.nvfp4_reconstruct_planes(p16.codes.cpu().numpy(), p16.scales.cpu().numpy(),
+                                            np.float32(st.item()), [n])
+    rec32 = oracle.mxfp4_reconstruct_planes(p32.codes.cpu().numpy(), p32.scales.cpu().numpy(), [n])
+    assert np.mean((rec16 - ref) ** 2) < np.mean((rec32 - ref) ** 2)
