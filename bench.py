@@ -170,10 +170,11 @@ class DecodeWorkload:
     a step appends one token at slot L0 (the same slot every visit, so every
     step attends exactly L0 + 1 tokens) and runs decode attention."""
 
-    def __init__(self, w, L0, replicas, with_append=True):
+    def __init__(self, w, L0, replicas, with_append=True, paged=False):
         import bit_decode_attention_b200 as nv
         self.nv = nv
-        self.w, self.L0, self.R, self.with_append = w, L0, replicas, with_append
+        assert not (paged and with_append), "the timed append writes contiguous planes"
+        self.w, self.L0, self.R, self.with_append, self.paged = w, L0, replicas, with_append, paged
         B, Hq, Hkv, D = w.B, w.Hq, w.Hkv, w.D
         self.S_max = synthetic.capacity(L0 + 1)
         dev = "cuda"
@@ -238,8 +239,30 @@ class DecodeWorkload:
         self.lens = torch.full((B,), L0 + 1 if with_append else L0, dtype=torch.int32, device=dev)
         self.ws = nv.new_workspace(B, Hq, Hkv, D)
         self.L_att = L0 + 1 if with_append else L0
+        if paged:
+            self._page_replicas(nv)
         torch.cuda.synchronize()
         assert self.status.item() == 0, "device status %d during set-up" % self.status.item()
+
+    def _page_replicas(self, nv, P=128):
+        """Move every replica cache into a pool of 128-token pages handed out in a
+        shuffled order (a seeded block table per replica, shared by K and V)."""
+        B, H = self.w.B, self.w.Hkv
+        M = (self.S_max + P - 1) // P
+        g = torch.Generator().manual_seed(7)
+        for r in range(self.R):
+            table = torch.randperm(B * M, generator=g).to(torch.int32).view(B, M).cuda()
+            planes = []
+            for pl in (self.k[r], self.v[r]):
+                pools = []
+                for t in (pl.codes, pl.scales):
+                    x = torch.nn.functional.pad(t, (0, 0, 0, M * P - self.S_max))
+                    x = x.view(B, H, M, P, -1).permute(0, 2, 1, 3, 4).reshape(B * M, H, P, -1)
+                    pool = torch.empty_like(x)
+                    pool[table.view(-1).long()] = x
+                    pools.append(pool)
+                planes.append(nv.PagedKVPlane(pools[0], pools[1], table))
+            self.k[r], self.v[r] = planes
 
     # kernels per step (ours): 1 append of K and V + 1 attention
     @property
@@ -264,8 +287,9 @@ class DecodeWorkload:
                                            self.k[r], self.v[r], status=self.status)
         if events is not None:
             events[0].record()
-        nv.nvfp4_decode_attention(self.q[r], self.k[r], self.v[r], self.sk, self.sv, self.lens,
-                                  out=self.out[r], workspace=self.ws, status=self.status)
+        attend = nv.nvfp4_decode_attention_paged if self.paged else nv.nvfp4_decode_attention
+        attend(self.q[r], self.k[r], self.v[r], self.sk, self.sv, self.lens,
+               out=self.out[r], workspace=self.ws, status=self.status)
         if events is not None:
             events[1].record()
 
@@ -585,6 +609,19 @@ def main():
             "frac_of_nominal_8tbs": ach / 8000.0 if ach else None, "steps": n_aux,
             "replicas": lwl.R}
         del lwl
+        torch.cuda.empty_cache()
+        # the gqa attention over a paged cache (128-token pages, shuffled block table)
+        gw = synthetic.get("gqa")
+        per = gw.B * gw.L * kv_bytes_per_token(gw.Hkv, gw.D)
+        pwl = DecodeWorkload(gw, gw.L, replicas_for(per, l2), with_append=False, paged=True)
+        pms, patt, pat_n, _ = time_decode(pwl, n_aux, 20, world, nvtx_name="timed_aux_paged")
+        pach = pwl.attention_bytes() / (patt / 1e3) / 1e9 if patt else None
+        aux["gqa_paged_attention"] = {
+            "workload": "gqa paged: B8 Hq32 Hkv8 D128 L4096, 128-token pages in shuffled order",
+            "kv_tokens_per_s": world * pwl.tokens_per_step() * n_aux / (pms / 1e3),
+            "launch_ms": patt, "achieved_gbs": pach, "frac_of_measured": pach / peak if pach else None,
+            "steps": n_aux, "replicas": pwl.R}
+        del pwl
         torch.cuda.empty_cache()
     line["aux"] = aux
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -28,6 +28,7 @@ __all__ = [
     "nvfp4_kv_dequant_fp8", "nvfp4_decode_attention_workspace", "nvfp4_decode_attention",
     "nvfp4_version", "NativeError", "nvfp4_decode_attention_noalloc",
     "mxfp4_cache_bytes", "mxfp4_kv_quantize_append",
+    "PagedKVPlane", "nvfp4_kv_quantize_append_paged", "nvfp4_decode_attention_paged",
 ]
 
 
@@ -87,6 +88,34 @@ class KVPlane:
         return _native.KVPlaneStruct(self.codes.data_ptr(), self.scales.data_ptr(), B, H, S, D)
 
 
+@dataclasses.dataclass
+class PagedKVPlane:
+    """One paged NVFP4 cache plane: a page pool and the block table.
+
+    codes       uint8 [num_pages][H_kv][page_tokens][D/2]
+    scales      uint8 [num_pages][H_kv][page_tokens][D/16]
+    block_table int32 [B][max_pages]; token t of sequence b lives in page
+                block_table[b][t // page_tokens], slot t % page_tokens
+    K and V planes of one cache share the block table.
+    """
+    codes: torch.Tensor
+    scales: torch.Tensor
+    block_table: torch.Tensor
+
+    @classmethod
+    def allocate(cls, num_pages: int, H_kv: int, page_tokens: int, D: int, block_table: torch.Tensor,
+                 device="cuda") -> "PagedKVPlane":
+        codes = torch.zeros(num_pages, H_kv, page_tokens, D // 2, dtype=torch.uint8, device=device)
+        scales = torch.zeros(num_pages, H_kv, page_tokens, D // 16, dtype=torch.uint8, device=device)
+        return cls(codes, scales, block_table)
+
+    def struct(self) -> _native.PagedPlaneStruct:
+        P, H, T, Dh = self.codes.shape
+        B, M = self.block_table.shape
+        return _native.PagedPlaneStruct(self.codes.data_ptr(), self.scales.data_ptr(),
+                                        self.block_table.data_ptr(), P, H, T, 2 * Dh, B, M)
+
+
 def nvfp4_version() -> str:
     return _native.lib().nvfp4_version().decode()
 
@@ -118,6 +147,18 @@ def nvfp4_kv_quantize_append(x_new: torch.Tensor, start_pos: torch.Tensor, s_ten
                                                 _ptr(start_pos), _ptr(new_lens), _ptr(s_tensor),
                                                 ctypes.byref(pl), _ptr(status), _stream(stream))
     _native.check("nvfp4_kv_quantize_append", st)
+
+
+def nvfp4_kv_quantize_append_paged(x_new: torch.Tensor, start_pos: torch.Tensor, s_tensor: torch.Tensor,
+                                   plane: PagedKVPlane, new_lens: Optional[torch.Tensor] = None,
+                                   status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """nvfp4_kv_quantize_append into a paged plane (slots found through its block table)."""
+    _need_cuda(x_new, start_pos, s_tensor, new_lens, status, plane.block_table)
+    pl = plane.struct()
+    st = _native.lib().nvfp4_kv_quantize_append_paged(_ptr(x_new), _dtype_code(x_new), x_new.shape[1],
+                                                      _ptr(start_pos), _ptr(new_lens), _ptr(s_tensor),
+                                                      ctypes.byref(pl), _ptr(status), _stream(stream))
+    _native.check("nvfp4_kv_quantize_append_paged", st)
 
 
 def nvfp4_kv_quantize_append_kv(x_k: torch.Tensor, x_v: torch.Tensor, start_pos: torch.Tensor,
@@ -203,6 +244,29 @@ def nvfp4_decode_attention(q: torch.Tensor, k: KVPlane, v: KVPlane, s_tensor_k: 
         _ptr(s_tensor_v), _ptr(seq_lens), ctypes.c_float(softmax_scale), _ptr(out),
         _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
     _native.check("nvfp4_decode_attention", st)
+    return out
+
+
+def nvfp4_decode_attention_paged(q: torch.Tensor, k: PagedKVPlane, v: PagedKVPlane,
+                                 s_tensor_k: torch.Tensor, s_tensor_v: torch.Tensor,
+                                 seq_lens: torch.Tensor, softmax_scale: float = 0.0,
+                                 out: Optional[torch.Tensor] = None,
+                                 workspace: Optional[torch.Tensor] = None,
+                                 status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """nvfp4_decode_attention over paged K/V planes that share one block table."""
+    _need_cuda(q, s_tensor_k, s_tensor_v, seq_lens, out, workspace, status, k.block_table)
+    B, H_q, D = q.shape
+    H_kv = k.codes.shape[1]
+    if out is None:
+        out = torch.empty(B, H_q, D, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(B, H_q, H_kv, D, device=q.device)
+    kp, vp = k.struct(), v.struct()
+    st = _native.lib().nvfp4_decode_attention_paged(
+        _ptr(q), _dtype_code(q), H_q, ctypes.byref(kp), ctypes.byref(vp), _ptr(s_tensor_k),
+        _ptr(s_tensor_v), _ptr(seq_lens), ctypes.c_float(softmax_scale), _ptr(out),
+        _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
+    _native.check("nvfp4_decode_attention_paged", st)
     return out
 
 

@@ -36,6 +36,8 @@ EXPORTS = (
     "nvfp4_decode_attention_noalloc",
     "mxfp4_cache_bytes",
     "mxfp4_kv_quantize_append",
+    "nvfp4_kv_quantize_append_paged",
+    "nvfp4_decode_attention_paged",
 )
 
 
@@ -48,6 +50,21 @@ class KVPlaneStruct(ctypes.Structure):
         ("H_kv", ctypes.c_int32),
         ("S_max", ctypes.c_int32),
         ("D", ctypes.c_int32),
+    ]
+
+
+class PagedPlaneStruct(ctypes.Structure):
+    """nvfp4_kv_paged_plane: host struct pointing at a device page pool and block table."""
+    _fields_ = [
+        ("codes", ctypes.c_void_p),
+        ("scales", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p),
+        ("num_pages", ctypes.c_int32),
+        ("H_kv", ctypes.c_int32),
+        ("page_tokens", ctypes.c_int32),
+        ("D", ctypes.c_int32),
+        ("B", ctypes.c_int32),
+        ("max_pages", ctypes.c_int32),
     ]
 
 
@@ -97,6 +114,12 @@ def lib():
     L.mxfp4_cache_bytes.restype = sz
     L.mxfp4_kv_quantize_append.argtypes = [vp, i32, i32, vp, vp, plane_p, vp, vp]
     L.mxfp4_kv_quantize_append.restype = i32
+    paged_p = ctypes.POINTER(PagedPlaneStruct)
+    L.nvfp4_kv_quantize_append_paged.argtypes = [vp, i32, i32, vp, vp, vp, paged_p, vp, vp]
+    L.nvfp4_kv_quantize_append_paged.restype = i32
+    L.nvfp4_decode_attention_paged.argtypes = [vp, i32, i32, paged_p, paged_p, vp, vp, vp, f32, vp, vp,
+                                               sz, vp, vp]
+    L.nvfp4_decode_attention_paged.restype = i32
     _lib = L
     return L
 

@@ -55,6 +55,87 @@ bool plane_ok(const nvfp4_kv_plane* pl) {
 
 nvfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
 
+bool paged_ok(const nvfp4_kv_paged_plane* pl) {
+    if (pl == nullptr || pl->codes == nullptr || pl->scales == nullptr || pl->block_table == nullptr)
+        return false;
+    if (pl->B < 0 || pl->H_kv <= 0 || pl->num_pages <= 0 || pl->max_pages <= 0) return false;
+    if (pl->page_tokens <= 0 || (pl->page_tokens % 128) != 0) return false;
+    if ((int64_t)pl->max_pages * pl->page_tokens > (int64_t)INT32_MAX) return false;
+    if (pl->D != 64 && pl->D != 128) return false;
+    if (!aligned16(pl->codes) || !aligned16(pl->scales)) return false;
+    return true;
+}
+
+// What a launch over sequences b0.. reads: contiguous planes advance by a
+// sequence stride; paged planes keep their pools and advance the block table.
+struct CacheView {
+    const uint8_t *kc, *ks, *vc, *vs;
+    size_t seq_code_bytes, seq_scale_bytes;
+    const int32_t* block_table;
+    int page_tokens, max_pages, num_pages;
+};
+
+// Validation and batch-chunked launches shared by the contiguous and the
+// paged attention entry points (the planes are already validated).
+nvfp4_status run_attention(const void* q, nvfp4_dtype q_dtype, int H_q, int B, int H_kv, int D,
+                           int S_max, const CacheView& c, const float* d_s_tensor_k,
+                           const float* d_s_tensor_v, const int32_t* d_seq_lens, float softmax_scale,
+                           float* out, void* workspace, size_t workspace_bytes, int32_t* d_status,
+                           nvfp4_stream_t stream) {
+    if (q_dtype != NVFP4_IN_BF16 && q_dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
+    if (H_q <= 0 || (H_q % H_kv) != 0) return NVFP4_ERR_INVALID_ARG;
+    if (H_q / H_kv > 16) return NVFP4_ERR_UNSUPPORTED;
+    if (d_s_tensor_k == nullptr || d_s_tensor_v == nullptr || d_seq_lens == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!(std::isfinite(softmax_scale)) || softmax_scale < 0.0f) return NVFP4_ERR_INVALID_ARG;
+    if (B == 0) return NVFP4_OK;
+    if (q == nullptr || out == nullptr || !aligned16(q) || !aligned16(out)) return NVFP4_ERR_INVALID_ARG;
+    // the kernels split a launch's tiles (32 tokens at the smallest) of every
+    // (sequence, KV head) with 32-bit prefix sums
+    const int64_t launch_tiles = (int64_t)(B < kMaxBatchPerLaunch ? B : kMaxBatchPerLaunch) * H_kv *
+                                 (((int64_t)S_max + 31) / 32);
+    if (launch_tiles > (int64_t)INT32_MAX) return NVFP4_ERR_UNSUPPORTED;
+    const AttnWorkspace ws = attention_workspace(B, H_q, H_kv, D);
+    if (workspace == nullptr || workspace_bytes < ws.total_bytes || !aligned16(workspace))
+        return NVFP4_ERR_WORKSPACE;
+
+    const size_t esz = q_dtype == NVFP4_IN_F32 ? 4 : 2;
+    AttnLaunch a{};
+    a.q_f32 = q_dtype == NVFP4_IN_F32;
+    a.Hq = H_q;
+    a.Hkv = H_kv;
+    a.S_max = S_max;
+    a.D = D;
+    a.st_k = d_s_tensor_k;
+    a.st_v = d_s_tensor_v;
+    a.softmax_scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt((float)D);
+    a.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ws.counters_bytes);
+    a.status = d_status;
+    a.grid = ws.grid;
+    a.block_table = c.block_table;
+    a.page_tokens = c.page_tokens;
+    a.max_pages = c.max_pages;
+    a.num_pages = c.num_pages;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    for (int b0 = 0; b0 < B; b0 += kMaxBatchPerLaunch) {
+        const int nb = (B - b0) < kMaxBatchPerLaunch ? (B - b0) : kMaxBatchPerLaunch;
+        a.B = nb;
+        a.q = static_cast<const uint8_t*>(q) + (size_t)b0 * H_q * D * esz;
+        a.kc = c.kc + (size_t)b0 * c.seq_code_bytes;    // paged: offsets 0, the table moves
+        a.ks = c.ks + (size_t)b0 * c.seq_scale_bytes;
+        a.vc = c.vc + (size_t)b0 * c.seq_code_bytes;
+        a.vs = c.vs + (size_t)b0 * c.seq_scale_bytes;
+        if (c.block_table != nullptr) a.block_table = c.block_table + (size_t)b0 * c.max_pages;
+        a.seq_lens = d_seq_lens + b0;
+        a.out = out + (size_t)b0 * H_q * D;
+        a.counters = static_cast<int32_t*>(workspace) + (size_t)b0 * H_kv;
+        cudaError_t e = launch_decode_attention(a, s);
+        if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_OK;
+}
+
+
 }  // namespace
 
 extern "C" {
@@ -103,6 +184,22 @@ nvfp4_status nvfp4_kv_quantize_append(const void* x_new, nvfp4_dtype dtype, int 
     return from_cuda(launch_quantize_append(x_new, dtype == NVFP4_IN_F32, n_new, d_start_pos,
                                             d_new_lens, d_s_tensor, *plane, d_status,
                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_kv_quantize_append_paged(const void* x_new, nvfp4_dtype dtype, int n_new,
+                                            const int32_t* d_start_pos, int32_t* d_new_lens,
+                                            const float* d_s_tensor,
+                                            const nvfp4_kv_paged_plane* plane, int32_t* d_status,
+                                            nvfp4_stream_t stream) {
+    if (!paged_ok(plane) || n_new < 0 || d_s_tensor == nullptr || d_start_pos == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (dtype != NVFP4_IN_BF16 && dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
+    if (d_new_lens != nullptr && d_new_lens == d_start_pos) return NVFP4_ERR_INVALID_ARG;
+    if (n_new == 0 || plane->B == 0) return NVFP4_OK;
+    if (x_new == nullptr || !aligned16(x_new)) return NVFP4_ERR_INVALID_ARG;
+    return from_cuda(launch_quantize_append_paged(x_new, dtype == NVFP4_IN_F32, n_new, d_start_pos,
+                                                  d_new_lens, d_s_tensor, *plane, d_status,
+                                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
 nvfp4_status nvfp4_kv_quantize_append_kv(const void* x_k, const void* x_v, nvfp4_dtype dtype,
@@ -169,55 +266,35 @@ nvfp4_status nvfp4_decode_attention(const void* q, nvfp4_dtype q_dtype, int H_q,
     if (!plane_ok(k) || !plane_ok(v)) return NVFP4_ERR_INVALID_ARG;
     if (k->B != v->B || k->H_kv != v->H_kv || k->S_max != v->S_max || k->D != v->D)
         return NVFP4_ERR_INVALID_ARG;
-    if (q_dtype != NVFP4_IN_BF16 && q_dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
-    if (H_q <= 0 || (H_q % k->H_kv) != 0) return NVFP4_ERR_INVALID_ARG;
-    if (H_q / k->H_kv > 16) return NVFP4_ERR_UNSUPPORTED;
-    if (d_s_tensor_k == nullptr || d_s_tensor_v == nullptr || d_seq_lens == nullptr)
-        return NVFP4_ERR_INVALID_ARG;
-    if (!(std::isfinite(softmax_scale)) || softmax_scale < 0.0f) return NVFP4_ERR_INVALID_ARG;
-    const int B = k->B;
-    if (B == 0) return NVFP4_OK;
-    if (q == nullptr || out == nullptr || !aligned16(q) || !aligned16(out)) return NVFP4_ERR_INVALID_ARG;
-    // the kernels split a launch's tiles (32 tokens at the smallest) of every
-    // (sequence, KV head) with 32-bit prefix sums
-    const int64_t launch_tiles = (int64_t)(B < kMaxBatchPerLaunch ? B : kMaxBatchPerLaunch) * k->H_kv *
-                                 (((int64_t)k->S_max + 31) / 32);
-    if (launch_tiles > (int64_t)INT32_MAX) return NVFP4_ERR_UNSUPPORTED;
-    const AttnWorkspace ws = attention_workspace(B, H_q, k->H_kv, k->D);
-    if (workspace == nullptr || workspace_bytes < ws.total_bytes || !aligned16(workspace))
-        return NVFP4_ERR_WORKSPACE;
-
-    const int D = k->D;
-    const size_t esz = q_dtype == NVFP4_IN_F32 ? 4 : 2;
+    CacheView c{};
+    c.kc = k->codes; c.ks = k->scales; c.vc = v->codes; c.vs = v->scales;
     const size_t plane_tok = (size_t)k->H_kv * k->S_max;  // token slots per sequence
-    AttnLaunch a{};
-    a.q_f32 = q_dtype == NVFP4_IN_F32;
-    a.Hq = H_q;
-    a.Hkv = k->H_kv;
-    a.S_max = k->S_max;
-    a.D = D;
-    a.st_k = d_s_tensor_k;
-    a.st_v = d_s_tensor_v;
-    a.softmax_scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt((float)D);
-    a.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ws.counters_bytes);
-    a.status = d_status;
-    a.grid = ws.grid;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    for (int b0 = 0; b0 < B; b0 += kMaxBatchPerLaunch) {
-        const int nb = (B - b0) < kMaxBatchPerLaunch ? (B - b0) : kMaxBatchPerLaunch;
-        a.B = nb;
-        a.q = static_cast<const uint8_t*>(q) + (size_t)b0 * H_q * D * esz;
-        a.kc = k->codes + (size_t)b0 * plane_tok * (D / 2);
-        a.ks = k->scales + (size_t)b0 * plane_tok * (D / 16);
-        a.vc = v->codes + (size_t)b0 * plane_tok * (D / 2);
-        a.vs = v->scales + (size_t)b0 * plane_tok * (D / 16);
-        a.seq_lens = d_seq_lens + b0;
-        a.out = out + (size_t)b0 * H_q * D;
-        a.counters = static_cast<int32_t*>(workspace) + (size_t)b0 * k->H_kv;
-        cudaError_t e = launch_decode_attention(a, s);
-        if (e != cudaSuccess) return NVFP4_ERR_CUDA;
-    }
-    return NVFP4_OK;
+    c.seq_code_bytes = plane_tok * (k->D / 2);
+    c.seq_scale_bytes = plane_tok * (k->D / 16);
+    return run_attention(q, q_dtype, H_q, k->B, k->H_kv, k->D, k->S_max, c, d_s_tensor_k, d_s_tensor_v,
+                         d_seq_lens, softmax_scale, out, workspace, workspace_bytes, d_status, stream);
+}
+
+nvfp4_status nvfp4_decode_attention_paged(const void* q, nvfp4_dtype q_dtype, int H_q,
+                                          const nvfp4_kv_paged_plane* k,
+                                          const nvfp4_kv_paged_plane* v,
+                                          const float* d_s_tensor_k, const float* d_s_tensor_v,
+                                          const int32_t* d_seq_lens, float softmax_scale,
+                                          float* out, void* workspace, size_t workspace_bytes,
+                                          int32_t* d_status, nvfp4_stream_t stream) {
+    if (!paged_ok(k) || !paged_ok(v)) return NVFP4_ERR_INVALID_ARG;
+    if (k->block_table != v->block_table || k->B != v->B || k->H_kv != v->H_kv ||
+        k->page_tokens != v->page_tokens || k->max_pages != v->max_pages || k->D != v->D)
+        return NVFP4_ERR_INVALID_ARG;
+    CacheView c{};
+    c.kc = k->codes; c.ks = k->scales; c.vc = v->codes; c.vs = v->scales;
+    c.block_table = k->block_table;
+    c.page_tokens = k->page_tokens;
+    c.max_pages = k->max_pages;
+    c.num_pages = k->num_pages < v->num_pages ? k->num_pages : v->num_pages;
+    return run_attention(q, q_dtype, H_q, k->B, k->H_kv, k->D, k->max_pages * k->page_tokens, c,
+                         d_s_tensor_k, d_s_tensor_v, d_seq_lens, softmax_scale, out, workspace,
+                         workspace_bytes, d_status, stream);
 }
 
 }  // extern "C"

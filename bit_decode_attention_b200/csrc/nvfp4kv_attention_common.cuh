@@ -31,6 +31,11 @@ struct Params {
     int32_t* status;
     int B, Hq, Hkv, g, S_max;
     float softmax_scale;
+    // paged cache (block_table != nullptr): token t of sequence b sits in page
+    // block_table[b * max_pages + t / page_tokens], slot t % page_tokens, of a
+    // pool laid out [page][Hkv][page_tokens][...]; S_max = max_pages * page_tokens
+    const int32_t* block_table;
+    int page_tokens, max_pages, num_pages;
 };
 
 // Global tile index -> (sequence, head, first tile of the unit, length).
@@ -95,7 +100,20 @@ __device__ __forceinline__ void issue_tile(const Params& p, const Unit& u, int64
     const uint32_t scale_bytes = (uint32_t)ncopy * SB;
     mbar_arrive_expect_tx(bar, 2 * (code_bytes + scale_bytes));
     if (ncopy > 0) {
-        const int64_t tok = ((int64_t)u.b * p.Hkv + u.h) * p.S_max + t0;
+        int64_t tok;
+        if (p.block_table == nullptr) {
+            tok = ((int64_t)u.b * p.Hkv + u.h) * p.S_max + t0;
+        } else {
+            // a tile never straddles two pages (page_tokens is a multiple of
+            // 128, a multiple of every tile size); an entry outside the pool is
+            // reported and read from page 0, so no copy leaves the pool
+            int page = __ldg(p.block_table + (int64_t)u.b * p.max_pages + t0 / p.page_tokens);
+            if (page < 0 || page >= p.num_pages) {
+                report(p.status, NVFP4_ERR_INVALID_ARG);
+                page = 0;
+            }
+            tok = ((int64_t)page * p.Hkv + u.h) * p.page_tokens + t0 % p.page_tokens;
+        }
         bulk_g2s(stage, p.kc + tok * KB, code_bytes, bar);
         bulk_g2s(stage + OFF_VC, p.vc + tok * KB, code_bytes, bar);
         bulk_g2s(stage + OFF_KS, p.ks + tok * SB, scale_bytes, bar);

@@ -713,6 +713,10 @@ cudaError_t launch_decode_attention(const AttnLaunch& a, cudaStream_t stream) {
     p.status = a.status;
     p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.g = a.Hq / a.Hkv; p.S_max = a.S_max;
     p.softmax_scale = a.softmax_scale;
+    p.block_table = a.block_table;
+    p.page_tokens = a.page_tokens;
+    p.max_pages = a.max_pages;
+    p.num_pages = a.num_pages;
     const bool two = p.g > 8;
     const int sms = device_sm_count();
     if (a.D == 128 && !a.q_f32)   // fifth-generation tensor cores: the main path

@@ -211,12 +211,16 @@ __global__ void __launch_bounds__(256) quantize_append_kv_kernel(
     }
 }
 
+// With a block table (paged planes), token slot `pos` of sequence b is slot
+// pos % page_tokens of pool page block_table[b * max_pages + pos / page_tokens]
+// (pool layout [page][Hkv][page_tokens][...]) and S_max = max_pages * page_tokens.
 template <bool F32>
 __global__ void __launch_bounds__(256) quantize_append_kernel(
     const void* __restrict__ x_new, int B, int n_new, int Hkv, int D,
     const int32_t* __restrict__ start_pos, int32_t* __restrict__ new_lens,
     const float* __restrict__ s_tensor_p, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-    int S_max, int32_t* __restrict__ status) {
+    int S_max, int32_t* __restrict__ status, const int32_t* __restrict__ block_table, int page_tokens,
+    int max_pages, int num_pages) {
     const int nblk = D / 16;
     const int64_t total = (int64_t)B * Hkv * n_new * nblk;
     const float st = *s_tensor_p;
@@ -240,11 +244,22 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(
             continue;
         }
         if (leader && new_lens != nullptr) new_lens[b] = start + n_new;
+        int64_t slot;
+        if (block_table == nullptr) {
+            slot = ((int64_t)b * Hkv + h) * S_max + start + t;
+        } else {
+            const int pos = start + t;
+            const int page = block_table[(int64_t)b * max_pages + pos / page_tokens];
+            if (page < 0 || page >= num_pages) {
+                report(status, NVFP4_ERR_INVALID_ARG);
+                continue;
+            }
+            slot = ((int64_t)page * Hkv + h) * page_tokens + pos % page_tokens;
+        }
         float v[16];
         load16<F32>(x_new, (((int64_t)b * n_new + t) * Hkv + h) * D + 16 * blk, v);
         uint2 packed;
         const uint32_t sb = quantize_block(v, st, packed);
-        const int64_t slot = ((int64_t)b * Hkv + h) * S_max + start + t;
         *reinterpret_cast<uint2*>(codes + slot * (D / 2) + 8 * blk) = packed;
         scales[slot * (D / 16) + blk] = (uint8_t)sb;
     }
@@ -381,11 +396,33 @@ cudaError_t launch_quantize_append(const void* x_new, bool f32, int n_new,
     if (f32)
         quantize_append_kernel<true><<<(int)grid, threads, 0, stream>>>(
             x_new, pl.B, n_new, pl.H_kv, pl.D, d_start_pos, d_new_lens, d_s_tensor, pl.codes,
-            pl.scales, pl.S_max, d_status);
+            pl.scales, pl.S_max, d_status, nullptr, 0, 0, 0);
     else
         quantize_append_kernel<false><<<(int)grid, threads, 0, stream>>>(
             x_new, pl.B, n_new, pl.H_kv, pl.D, d_start_pos, d_new_lens, d_s_tensor, pl.codes,
-            pl.scales, pl.S_max, d_status);
+            pl.scales, pl.S_max, d_status, nullptr, 0, 0, 0);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_append_paged(const void* x_new, bool f32, int n_new,
+                                         const int32_t* d_start_pos, int32_t* d_new_lens,
+                                         const float* d_s_tensor, const nvfp4_kv_paged_plane& pp,
+                                         int32_t* d_status, cudaStream_t stream) {
+    const int64_t total = (int64_t)pp.B * pp.H_kv * n_new * (pp.D / 16);
+    if (total == 0) return cudaSuccess;
+    const int threads = 256;
+    int64_t grid = (total + threads - 1) / threads;
+    const int64_t cap = 16L * device_sm_count();
+    if (grid > cap) grid = cap;
+    const int S_max = pp.max_pages * pp.page_tokens;   // fits: checked by the caller
+    if (f32)
+        quantize_append_kernel<true><<<(int)grid, threads, 0, stream>>>(
+            x_new, pp.B, n_new, pp.H_kv, pp.D, d_start_pos, d_new_lens, d_s_tensor, pp.codes,
+            pp.scales, S_max, d_status, pp.block_table, pp.page_tokens, pp.max_pages, pp.num_pages);
+    else
+        quantize_append_kernel<false><<<(int)grid, threads, 0, stream>>>(
+            x_new, pp.B, n_new, pp.H_kv, pp.D, d_start_pos, d_new_lens, d_s_tensor, pp.codes,
+            pp.scales, S_max, d_status, pp.block_table, pp.page_tokens, pp.max_pages, pp.num_pages);
     return cudaGetLastError();
 }
 

@@ -30,6 +30,10 @@ __host__ __device__ constexpr int64_t partial_slot_floats(int g, int D) {
 cudaError_t launch_calib(const void* x, bool f32, int64_t n, float* d_s_tensor, int32_t* d_status,
                          cudaStream_t stream);
 
+cudaError_t launch_quantize_append_paged(const void* x_new, bool f32, int n_new,
+                                         const int32_t* d_start_pos, int32_t* d_new_lens,
+                                         const float* d_s_tensor, const nvfp4_kv_paged_plane& pp,
+                                         int32_t* d_status, cudaStream_t stream);
 cudaError_t launch_mxfp4_quantize_append(const void* x_new, bool f32, int n_new,
                                          const int32_t* d_start_pos, int32_t* d_new_lens,
                                          const nvfp4_kv_plane& pl, int32_t* d_status,
@@ -62,6 +66,9 @@ struct AttnLaunch {
     int32_t* counters;   // [B * Hkv], zero between calls
     int32_t* status;
     int grid;            // CTAs
+    // paged cache: nullptr for contiguous planes (then S_max is the capacity)
+    const int32_t* block_table;
+    int page_tokens, max_pages, num_pages;
 };
 
 cudaError_t launch_decode_attention(const AttnLaunch& a, cudaStream_t stream);

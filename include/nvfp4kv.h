@@ -95,6 +95,30 @@ typedef struct {
     int32_t D;        /* head_dim, 64 or 128 */
 } nvfp4_kv_plane;
 
+/* One paged NVFP4 cache plane ([NVFP4-KV] "学術研究との関連": vLLM's
+ * PagedAttention block management is orthogonal to the NVFP4 cache and
+ * combines with it).  A pool of pages, each holding page_tokens token slots
+ * of every KV head, and a block table that maps (sequence, logical page) to a
+ * pool page.  The struct lives in host memory; the arrays in device memory.
+ *   codes       uint8 [num_pages][H_kv][page_tokens][D/2], 16-byte aligned
+ *   scales      uint8 [num_pages][H_kv][page_tokens][D/16], 16-byte aligned
+ *   block_table int32 [B][max_pages]: token t of sequence b lives in pool page
+ *               block_table[b * max_pages + t / page_tokens], slot
+ *               t % page_tokens; entries past a sequence's length are unread
+ * Element encoding, packing and scales are those of nvfp4_kv_plane.  The
+ * capacity of a sequence is max_pages * page_tokens tokens. */
+typedef struct {
+    uint8_t* codes;
+    uint8_t* scales;
+    const int32_t* block_table;
+    int32_t num_pages;    /* pages in the pool, >= 1 */
+    int32_t H_kv;         /* KV heads */
+    int32_t page_tokens;  /* token slots per page, a multiple of 128 */
+    int32_t D;            /* head_dim, 64 or 128 */
+    int32_t B;            /* sequences (rows of the block table) */
+    int32_t max_pages;    /* block-table entries per sequence, >= 1 */
+} nvfp4_kv_paged_plane;
+
 /* Human-readable name of a status value (static string). */
 const char* nvfp4_status_string(int status);
 
@@ -161,6 +185,17 @@ nvfp4_status mxfp4_kv_quantize_append(const void* x_new, nvfp4_dtype dtype, int 
                                       const nvfp4_kv_plane* plane, int32_t* d_status,
                                       nvfp4_stream_t stream);
 
+/* nvfp4_kv_quantize_append into a paged plane: the slot of token t of
+ * sequence b is found through the block table.  Capacity errors as for
+ * contiguous planes (start + n_new > max_pages * page_tokens); a block-table
+ * entry outside [0, num_pages) skips that token's blocks and reports
+ * NVFP4_ERR_INVALID_ARG through *d_status. */
+nvfp4_status nvfp4_kv_quantize_append_paged(const void* x_new, nvfp4_dtype dtype, int n_new,
+                                            const int32_t* d_start_pos, int32_t* d_new_lens,
+                                            const float* d_s_tensor,
+                                            const nvfp4_kv_paged_plane* plane, int32_t* d_status,
+                                            nvfp4_stream_t stream);
+
 /* Quantize-append the same new tokens into the K and the V plane in one
  * launch ([NVFP4-KV] "量子化・逆量子化フロー": K and V are both quantized
  * on append).  Same results, arguments and errors as two calls of
@@ -213,6 +248,21 @@ nvfp4_status nvfp4_decode_attention(const void* q, nvfp4_dtype q_dtype, int H_q,
                                     const int32_t* d_seq_lens, float softmax_scale,
                                     float* out, void* workspace, size_t workspace_bytes,
                                     int32_t* d_status, nvfp4_stream_t stream);
+
+/* nvfp4_decode_attention over paged K and V planes.  k and v share one block
+ * table (the same pointer) and agree in B, H_kv, page_tokens, max_pages, D;
+ * their pools may differ.  Arguments, results and errors are those of
+ * nvfp4_decode_attention with S_max = max_pages * page_tokens; the workspace
+ * size is nvfp4_decode_attention_workspace(B, H_q, H_kv, D).  A block-table
+ * entry outside [0, num_pages) is reported as NVFP4_ERR_INVALID_ARG through
+ * *d_status and page 0 is read in its place (no access leaves the pool). */
+nvfp4_status nvfp4_decode_attention_paged(const void* q, nvfp4_dtype q_dtype, int H_q,
+                                          const nvfp4_kv_paged_plane* k,
+                                          const nvfp4_kv_paged_plane* v,
+                                          const float* d_s_tensor_k, const float* d_s_tensor_v,
+                                          const int32_t* d_seq_lens, float softmax_scale,
+                                          float* out, void* workspace, size_t workspace_bytes,
+                                          int32_t* d_status, nvfp4_stream_t stream);
 
 /* Decode attention for callers that cannot allocate device memory.
  *

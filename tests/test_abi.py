@@ -124,6 +124,29 @@ def test_argument_validation_without_gpu(lib):
     assert mx(ctypes.c_void_p(72), 0, 1, dev, None, ctypes.byref(mxp), None, None) == INVALID
     assert mx(dev, 0, 1, None, None, ctypes.byref(mxp), None, None) == INVALID      # no start
     assert mx(dev, 0, 0, dev, None, ctypes.byref(mxp), None, None) == 0             # no-op
+    # paged planes: page_tokens a multiple of 128, a block table, a shared table for K and V
+    PP = _native.PagedPlaneStruct
+    tbl = ctypes.c_void_p(256)
+    pg = PP(16, 16, tbl, 4, 2, 128, 128, 2, 3)
+    pg_other = PP(16, 16, ctypes.c_void_p(512), 4, 2, 128, 128, 2, 3)
+    bad_pages = [PP(16, 16, tbl, 4, 2, 96, 128, 2, 3),      # page not a multiple of 128
+                 PP(16, 16, None, 4, 2, 128, 128, 2, 3),     # no block table
+                 PP(16, 16, tbl, 0, 2, 128, 128, 2, 3),      # empty pool
+                 PP(16, 16, tbl, 4, 2, 128, 96, 2, 3),       # head_dim
+                 PP(16, 16, tbl, 4, 2, 1 << 24, 128, 2, 1 << 10),   # capacity past 2^31
+                 PP(17, 16, tbl, 4, 2, 128, 128, 2, 3)]      # misaligned codes
+    qp = lib.nvfp4_kv_quantize_append_paged
+    for bp in bad_pages:
+        assert qp(dev, 0, 1, dev, None, dev, ctypes.byref(bp), None, None) == INVALID
+    assert qp(dev, 0, 1, dev, None, None, ctypes.byref(pg), None, None) == INVALID     # no scale
+    assert qp(dev, 0, 0, dev, None, dev, ctypes.byref(pg), None, None) == 0            # no-op
+    ap = lib.nvfp4_decode_attention_paged
+    pargs = lambda kk, vv, ws, nbytes: (dev, 0, 4, ctypes.byref(kk), ctypes.byref(vv), dev, dev, dev,
+                                        ctypes.c_float(0.0), dev, ws, nbytes, None, None)
+    for bp in bad_pages:
+        assert ap(*pargs(bp, bp, dev, 1 << 30)) == INVALID
+    assert ap(*pargs(pg, pg_other, dev, 1 << 30)) == INVALID     # K and V tables differ
+    assert ap(*pargs(pg, pg, dev, 16)) == WS
     cal = lib.nvfp4_calib_tensor_scale
     assert cal(dev, 0, -1, dev, None, None) == INVALID
     assert cal(dev, 0, 10, None, None, None) == INVALID

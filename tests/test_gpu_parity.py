@@ -375,3 +375,113 @@ def test_mxfp4_error_above_nvfp4_on_device_codes(nv):
                                             np.float32(st.item()), [n])
     rec32 = oracle.mxfp4_reconstruct_planes(p32.codes.cpu().numpy(), p32.scales.cpu().numpy(), [n])
     assert np.mean((rec16 - ref) ** 2) < np.mean((rec32 - ref) ** 2)
+
+
+# ---------------------------------------------------------------------------
+# Paged cache: a page pool and a block table in place of contiguous slabs
+# ---------------------------------------------------------------------------
+def _paged_setup(nv, B, H, D, page_tokens, max_pages, num_pages, seed):
+    """A block table that hands out distinct pool pages in a shuffled order."""
+    g = torch.Generator().manual_seed(seed)
+    perm = torch.randperm(num_pages, generator=g)[:B * max_pages]
+    table = perm.view(B, max_pages).to(torch.int32).cuda()
+    k = nv.PagedKVPlane.allocate(num_pages, H, page_tokens, D, table)
+    v = nv.PagedKVPlane.allocate(num_pages, H, page_tokens, D, table)
+    return table, k, v
+
+
+def _gather(plane, table_np, S):
+    """Contiguous [B][H][S][...] views of a paged plane, by following its table."""
+    codes, scales = plane.codes.cpu().numpy(), plane.scales.cpu().numpy()
+    B, M = table_np.shape
+    P = codes.shape[2]
+    oc = np.zeros((B, codes.shape[1], S, codes.shape[3]), np.uint8)
+    os_ = np.zeros((B, scales.shape[1], S, scales.shape[3]), np.uint8)
+    for b in range(B):
+        for m in range(S // P):
+            oc[b, :, m * P:(m + 1) * P] = codes[table_np[b, m]]
+            os_[b, :, m * P:(m + 1) * P] = scales[table_np[b, m]]
+    return oc, os_
+
+
+@pytest.mark.parametrize("D,q_dtype", [(128, "bf16"), (128, "f32"), (64, "bf16")])
+def test_paged_cache_matches_contiguous_and_oracle(nv, D, q_dtype):
+    B, H, Hq, P, M = 3, 2, 8, 128, 4
+    S = P * M
+    w = synthetic.shrink(synthetic.get("long64k"), B=B, Hq=Hq, Hkv=H, D=D)
+    table, kp, vp = _paged_setup(nv, B, H, D, P, M, 20, seed=D)
+    lens = [300, 129, 511]
+    xk = synthetic.kv_tokens(w, S, "k")
+    xv = synthetic.kv_tokens(w, S, "v")
+    sk = nv.nvfp4_calib_tensor_scale(to_dev(xk.reshape(-1), "bf16"))
+    sv = nv.nvfp4_calib_tensor_scale(to_dev(xv.reshape(-1), "bf16"))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    new_lens = torch.zeros(B, dtype=torch.int32, device="cuda")
+    # a prefill of 300 tokens, then the rest one chunk at a time: pages are crossed mid-append
+    for lo, hi in ((0, 300), (300, 301), (301, S)):
+        start = torch.full((B,), lo, dtype=torch.int32, device="cuda")
+        nv.nvfp4_kv_quantize_append_paged(to_dev(xk[:, lo:hi], "bf16"), start, sk, kp, new_lens=new_lens,
+                                          status=status)
+        nv.nvfp4_kv_quantize_append_paged(to_dev(xv[:, lo:hi], "bf16"), start, sv, vp, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0 and new_lens.tolist() == [S] * B
+    # the pages, read through the table, hold exactly the oracle's contiguous planes
+    table_np = table.cpu().numpy()
+    kc, ks = _gather(kp, table_np, S)
+    vc, vs = _gather(vp, table_np, S)
+    _, st_k = oracle.tensor_scale(xk.reshape(-1).numpy())
+    _, st_v = oracle.tensor_scale(xv.reshape(-1).numpy())
+    okc, oks = oracle.new_planes(B, H, S, D)
+    ovc, ovs = oracle.new_planes(B, H, S, D)
+    z = np.zeros(B, np.int32)
+    assert oracle.quantize_append(xk.numpy(), z, st_k, okc, oks) == 0
+    assert oracle.quantize_append(xv.numpy(), z, st_v, ovc, ovs) == 0
+    for got, want in ((kc, okc), (ks, oks), (vc, ovc), (vs, ovs)):
+        np.testing.assert_array_equal(got, want)
+    # attention through the table equals attention over the same bytes laid out contiguously
+    q = synthetic.queries(w)
+    qd = to_dev(q, q_dtype)
+    lens_d = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    paged = nv.nvfp4_decode_attention_paged(qd, kp, vp, sk, sv, lens_d, status=status)
+    kcont = nv.KVPlane(torch.from_numpy(kc).cuda(), torch.from_numpy(ks).cuda())
+    vcont = nv.KVPlane(torch.from_numpy(vc).cuda(), torch.from_numpy(vs).cuda())
+    cont = nv.nvfp4_decode_attention(qd, kcont, vcont, sk, sv, lens_d, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.equal(paged, cont)
+    want = oracle.decode_attention_nvfp4(q.numpy(), okc, oks, ovc, ovs, st_k, st_v, np.array(lens, np.int32))
+    assert_attention_close(paged.cpu().numpy(), want)
+
+
+def test_paged_bad_table_entries_are_reported(nv):
+    B, H, D, P, M, NP = 2, 1, 128, 128, 2, 4
+    table = torch.tensor([[0, 1], [2, 3]], dtype=torch.int32, device="cuda")
+    kp = nv.PagedKVPlane.allocate(NP, H, P, D, table)
+    vp = nv.PagedKVPlane.allocate(NP, H, P, D, table)
+    x = torch.ones(B, 200, H, D, device="cuda")
+    st = torch.tensor([0.01], device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_kv_quantize_append_paged(x, torch.zeros(B, dtype=torch.int32, device="cuda"), st, kp,
+                                      status=status)
+    nv.nvfp4_kv_quantize_append_paged(x, torch.zeros(B, dtype=torch.int32, device="cuda"), st, vp,
+                                      status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    # sequence 1's second page points outside the pool: appends skip it, attention
+    # reads page 0 in its place; both report the bad entry
+    bad = torch.tensor([[0, 1], [2, NP]], dtype=torch.int32, device="cuda")
+    kb = nv.PagedKVPlane(kp.codes, kp.scales, bad)
+    vb = nv.PagedKVPlane(vp.codes, vp.scales, bad)
+    before = kp.codes.clone()
+    nv.nvfp4_kv_quantize_append_paged(x[:, :1].contiguous(), torch.tensor([150, 150], dtype=torch.int32, device="cuda"),
+                                      st, kb, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == nv.NVFP4_ERR_INVALID_ARG
+    assert torch.equal(kp.codes[3], before[3])
+    status.zero_()
+    q = torch.ones(B, 4, D, dtype=torch.bfloat16, device="cuda")
+    out = nv.nvfp4_decode_attention_paged(q, kb, vb, st, st, torch.tensor([200, 200], dtype=torch.int32,
+                                                                          device="cuda"), status=status)
+    torch.cuda.synchronize()
+    assert status.item() == nv.NVFP4_ERR_INVALID_ARG
+    assert torch.isfinite(out).all()
