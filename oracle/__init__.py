@@ -68,6 +68,10 @@ def lib():
         L.oracle_mxfp4_quantize_append.restype = ctypes.c_int
         L.oracle_mxfp4_reconstruct_planes.argtypes = [u8p, u8p, ctypes.c_int, ctypes.c_int,
                                                       ctypes.c_int, ctypes.c_int, i32p, f64p]
+        L.oracle_prefill_attention_nvfp4.argtypes = [f32p, u8p, u8p, u8p, u8p, ctypes.c_float,
+                                                     ctypes.c_float, ctypes.c_int, ctypes.c_int,
+                                                     ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                     ctypes.c_int, i32p, ctypes.c_double, f64p]
         L.oracle_mxfp4_bits_per_element.argtypes = []
         L.oracle_mxfp4_bits_per_element.restype = ctypes.c_double
         L.oracle_kv_bytes.restype = ctypes.c_double
@@ -266,6 +270,24 @@ def decode_attention_nvfp4(q, k_codes, k_scales, v_codes, v_scales, s_tensor_k, 
         _p(c(v_codes), ctypes.c_uint8), _p(c(v_scales), ctypes.c_uint8),
         np.float32(s_tensor_k), np.float32(s_tensor_v), B, H_q, H_kv, S_max, D,
         _p(seq_lens, ctypes.c_int32), float(softmax_scale), _p(out, ctypes.c_double))
+    return out
+
+
+def prefill_attention_nvfp4(q, k_codes, k_scales, v_codes, v_scales, s_tensor_k, s_tensor_v,
+                            start, softmax_scale=0.0):
+    """q fp32 [B][C][H_q][D] at positions start[b] + i -> fp64 [B][C][H_q][D] (causal)."""
+    q = _f32(q)
+    B, C, H_q, D = q.shape
+    _, H_kv, S_max, _ = k_codes.shape
+    start = np.ascontiguousarray(start, np.int32)
+    assert np.all(start >= 0) and np.all(start + C <= S_max)
+    out = np.zeros((B, C, H_q, D), np.float64)
+    c = np.ascontiguousarray
+    lib().oracle_prefill_attention_nvfp4(
+        _p(q, ctypes.c_float), _p(c(k_codes), ctypes.c_uint8), _p(c(k_scales), ctypes.c_uint8),
+        _p(c(v_codes), ctypes.c_uint8), _p(c(v_scales), ctypes.c_uint8),
+        np.float32(s_tensor_k), np.float32(s_tensor_v), B, C, H_q, H_kv, S_max, D,
+        _p(start, ctypes.c_int32), float(softmax_scale), _p(out, ctypes.c_double))
     return out
 
 

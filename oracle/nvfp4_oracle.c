@@ -429,6 +429,55 @@ void oracle_decode_attention_nvfp4(const float* q,
 }
 
 /* --------------------------------------------------------------------------
+ * Chunked prefill over the cache.  [P1] and [P3] "推論速度" credit the NVFP4
+ * cache with a faster time to first token, which is the prefill side: the
+ * prompt is processed in chunks whose K/V are appended first, then each
+ * query of the chunk attends to the cache.  Reading R17: query i of sequence
+ * b sits at position start[b] + i and sees cache tokens t <= start[b] + i
+ * (causal), over the same FP8 values as decode attention (R7, R8); so each
+ * query is decode attention with its own length start[b] + i + 1.
+ * ------------------------------------------------------------------------ */
+void oracle_prefill_attention_nvfp4(const float* q,
+                                    const uint8_t* k_codes, const uint8_t* k_scales,
+                                    const uint8_t* v_codes, const uint8_t* v_scales,
+                                    float s_tensor_k, float s_tensor_v,
+                                    int B, int C, int H_q, int H_kv, int S_max, int D,
+                                    const int32_t* start, double softmax_scale, double* out) {
+    double scale = softmax_scale != 0.0 ? softmax_scale : 1.0 / sqrt((double)D);
+    int g = H_q / H_kv;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int hk = 0; hk < H_kv; ++hk) {
+            int L = start[b] + C;                     /* tokens any query of the chunk sees */
+            int64_t slot0 = ((int64_t)b * H_kv + hk) * S_max;
+            double* K = (double*)malloc(sizeof(double) * (size_t)L * D);
+            double* V = (double*)malloc(sizeof(double) * (size_t)L * D);
+            for (int t = 0; t < L; ++t) {
+                int64_t slot = slot0 + t;
+                for (int d = 0; d < D; ++d) {
+                    uint8_t kb = k_codes[slot * (D / 2) + d / 2];
+                    uint8_t vb = v_codes[slot * (D / 2) + d / 2];
+                    uint8_t kc = (d % 2 == 0) ? (kb & 0xF) : (kb >> 4);
+                    uint8_t vc = (d % 2 == 0) ? (vb & 0xF) : (vb >> 4);
+                    uint8_t ks = k_scales[slot * (D / 16) + d / 16];
+                    uint8_t vs = v_scales[slot * (D / 16) + d / 16];
+                    K[(int64_t)t * D + d] = oracle_e4m3_value(oracle_dequant_fp8(kc, ks, s_tensor_k));
+                    V[(int64_t)t * D + d] = oracle_e4m3_value(oracle_dequant_fp8(vc, vs, s_tensor_v));
+                }
+            }
+            for (int i = 0; i < C; ++i)
+                for (int j = 0; j < g; ++j) {
+                    int h = hk * g + j;
+                    int64_t row = (((int64_t)b * C + i) * H_q + h) * D;
+                    attend_one(q + row, K, V, start[b] + i + 1, D, scale, out + row);
+                }
+            free(K);
+            free(V);
+        }
+    }
+}
+
+/* --------------------------------------------------------------------------
  * Memory model.  [P3] "KV Cacheのメモリボトルネック": KV_mem = 2 * L * n_h *
  * d_h * s * b * sizeof(dtype).  For NVFP4 the per-element size is 4 code bits
  * plus one 8-bit scale shared by 16 elements ("E2M1 + 2レベルスケーリング");

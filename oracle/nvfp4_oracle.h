@@ -46,6 +46,8 @@
  *       one token; there is no tensor scale.
  *   R15 A block holding NaN or +-Inf gets the E8M0 NaN byte 0xFF and zero
  *       codes, and the append reports ORACLE_ERR_NONFINITE.
+ *   R17 Chunked prefill: query i of a chunk starting at position start sees
+ *       cache tokens 0..start+i (causal, its own K/V appended first).
  */
 #ifndef NVFP4_ORACLE_H
 #define NVFP4_ORACLE_H
@@ -138,6 +140,18 @@ void    oracle_mxfp4_reconstruct_planes(const uint8_t* codes, const uint8_t* sca
                                         int B, int H_kv, int S_max, int D,
                                         const int32_t* seq_lens, double* out);
 double  oracle_mxfp4_bits_per_element(void);
+
+/* ---- chunked prefill attention (reading R17), fp64 ----
+ * q     : fp32 [B][C][H_q][D], query i of sequence b at position start[b] + i
+ * start : int32 [B]; the caller guarantees start[b] + C <= S_max
+ * out   : fp64 [B][C][H_q][D]; query i attends to cache tokens
+ *         0 .. start[b] + i (its own K/V included), FP8 values as R7. */
+void    oracle_prefill_attention_nvfp4(const float* q,
+                                       const uint8_t* k_codes, const uint8_t* k_scales,
+                                       const uint8_t* v_codes, const uint8_t* v_scales,
+                                       float s_tensor_k, float s_tensor_v,
+                                       int B, int C, int H_q, int H_kv, int S_max, int D,
+                                       const int32_t* start, double softmax_scale, double* out);
 
 /* ---- memory model ([P3] "KV Cacheのメモリボトルネック") ----
  * KV bytes = 2 (K and V) * layers * n_h * s * b * bytes per head vector. */

@@ -84,6 +84,15 @@ MUTANTS = [
     ("mxfp4_scale_bias_wrong",
      "return ldexp(1.0, (int)byte - 127);", "return ldexp(1.0, (int)byte - 128);",
      [pins.test_e8m0_values]),
+    ("prefill_one_token_short",
+     "attend_one(q + row, K, V, start[b] + i + 1, D, scale, out + row);",
+     "attend_one(q + row, K, V, start[b] + i, D, scale, out + row);",
+     [pins.test_prefill_single_query_is_decode_attention,
+      pins.test_prefill_matches_torch_sdpa_with_causal_mask]),
+    ("prefill_query_positions_reversed",
+     "int64_t row = (((int64_t)b * C + i) * H_q + h) * D;",
+     "int64_t row = (((int64_t)b * C + (C - 1 - i)) * H_q + h) * D;",
+     [pins.test_prefill_matches_torch_sdpa_with_causal_mask, pins.test_prefill_is_causal]),
     ("nvfp4_reconstruction_without_tensor_scale",
      "oracle_e2m1_value(code) * oracle_e4m3_value(sb) * (double)s_tensor;",
      "oracle_e2m1_value(code) * oracle_e4m3_value(sb);",

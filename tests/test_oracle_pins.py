@@ -564,3 +564,63 @@ def test_mse_ordering_nvfp4_below_mxfp4():
     mse_nv = np.mean((oracle.nvfp4_reconstruct_planes(c16, s16, st, [n]) - ref) ** 2)
     mse_mx = np.mean((oracle.mxfp4_reconstruct_planes(c32, s32, [n]) - ref) ** 2)
     assert mse_nv < mse_mx
+
+
+# --------------------------------------------------------------------------
+# Chunked prefill over the cache (causal, reading R17)
+# --------------------------------------------------------------------------
+def _prefill_case(seed, B, C, H_q, H_kv, S, D):
+    rng = np.random.default_rng(seed)
+    x_k = rng.standard_normal((B, S, H_kv, D)).astype(np.float32)
+    x_v = rng.standard_normal((B, S, H_kv, D)).astype(np.float32)
+    _, sk = oracle.tensor_scale(x_k)
+    _, sv = oracle.tensor_scale(x_v)
+    kc, ks = oracle.new_planes(B, H_kv, S, D)
+    vc, vs = oracle.new_planes(B, H_kv, S, D)
+    zero = np.zeros(B, np.int32)
+    assert oracle.quantize_append(x_k, zero, sk, kc, ks) == 0
+    assert oracle.quantize_append(x_v, zero, sv, vc, vs) == 0
+    q = rng.standard_normal((B, C, H_q, D)).astype(np.float32)
+    return q, kc, ks, vc, vs, sk, sv
+
+
+def test_prefill_single_query_is_decode_attention():
+    q, kc, ks, vc, vs, sk, sv = _prefill_case(31, 3, 1, 4, 2, 48, 32)
+    start = np.array([0, 17, 47], np.int32)
+    got = oracle.prefill_attention_nvfp4(q, kc, ks, vc, vs, sk, sv, start)
+    want = oracle.decode_attention_nvfp4(q[:, 0], kc, ks, vc, vs, sk, sv, start + 1)
+    np.testing.assert_array_equal(got[:, 0], want)
+
+
+def test_prefill_matches_torch_sdpa_with_causal_mask():
+    B, C, H_q, H_kv, S, D = 2, 9, 6, 2, 40, 32
+    q, kc, ks, vc, vs, sk, sv = _prefill_case(37, B, C, H_q, H_kv, S, D)
+    start = np.array([0, 23], np.int32)
+    got = oracle.prefill_attention_nvfp4(q, kc, ks, vc, vs, sk, sv, start)
+    full = np.full(B, S, np.int32)
+    K = _fp8_values(oracle.dequant_planes(kc, ks, sk, full))
+    V = _fp8_values(oracle.dequant_planes(vc, vs, sv, full))
+    g = H_q // H_kv
+    for b in range(B):
+        L = int(start[b]) + C
+        qt = torch.from_numpy(q[b]).to(torch.float64).permute(1, 0, 2)          # [H_q][C][D]
+        Kt = K[b, :, :L].repeat_interleave(g, 0)
+        Vt = V[b, :, :L].repeat_interleave(g, 0)
+        pos = torch.arange(C)[:, None] + int(start[b])
+        mask = torch.arange(L)[None, :] <= pos                                   # [C][L]
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, attn_mask=mask)
+        np.testing.assert_allclose(got[b], ref.permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_is_causal():
+    B, C, H_q, H_kv, S, D = 1, 6, 2, 1, 32, 16
+    q, kc, ks, vc, vs, sk, sv = _prefill_case(41, B, C, H_q, H_kv, S, D)
+    start = np.array([10], np.int32)
+    base = oracle.prefill_attention_nvfp4(q, kc, ks, vc, vs, sk, sv, start)
+    # rewrite the K/V of position 13 (seen by queries 3.. of the chunk only)
+    kc2, vc2 = kc.copy(), vc.copy()
+    kc2[0, :, 13] ^= 0x77
+    vc2[0, :, 13] ^= 0x55
+    moved = oracle.prefill_attention_nvfp4(q, kc2, ks, vc2, vs, sk, sv, start)
+    np.testing.assert_array_equal(moved[0, :3], base[0, :3])
+    assert np.all(np.abs(moved[0, 3:] - base[0, 3:]).max(axis=(1, 2)) > 0)
