@@ -45,7 +45,7 @@ struct Unit {
 };
 
 template <int TILE = kTile>
-__device__ __forceinline__ Unit find_unit(const int32_t* prefix, const int32_t* lens, int B, int Hkv,
+__host__ __device__ __forceinline__ Unit find_unit(const int32_t* prefix, const int32_t* lens, int B, int Hkv,
                                           int64_t gt) {
     int lo = 0, hi = B;  // prefix[lo] <= gt < prefix[hi]
     while (hi - lo > 1) {
@@ -65,19 +65,19 @@ __device__ __forceinline__ Unit find_unit(const int32_t* prefix, const int32_t* 
 }
 
 // CTA c owns global tiles [range_start(c), range_start(c + 1)).
-__device__ __forceinline__ int64_t range_start(int64_t c, int64_t T, int64_t N) {
+__host__ __device__ __forceinline__ int64_t range_start(int64_t c, int64_t T, int64_t N) {
     return c * T / N;
 }
 
 // CTA owning global tile t when T tiles are cut into N equal ranges.
-__device__ __forceinline__ int64_t cta_of(int64_t t, int64_t T, int64_t N) {
+__host__ __device__ __forceinline__ int64_t cta_of(int64_t t, int64_t T, int64_t N) {
     return ((t + 1) * N - 1) / T;
 }
 
 // Partial-result slot of CTA cc for a unit starting at global tile U0: a CTA
 // can share at most two units with other CTAs -- the one holding its first
 // tile (slot 2cc) and the one holding its last tile (slot 2cc + 1).
-__device__ __forceinline__ int64_t partial_slot(int64_t cc, int64_t U0, int64_t T, int64_t N) {
+__host__ __device__ __forceinline__ int64_t partial_slot(int64_t cc, int64_t U0, int64_t T, int64_t N) {
     return (U0 <= range_start(cc, T, N)) ? 2 * cc : 2 * cc + 1;
 }
 
@@ -147,8 +147,20 @@ struct CombineSmem {
 // cta_of(U1 - 1) holds one; with T < N a non-empty range is a single tile,
 // so there is one CTA per tile.  (No loop over CTAs: a 64-bit division costs
 // a few hundred cycles, and the count sits on the critical path of the merge.)
-__device__ __forceinline__ int unit_contributors(int64_t U0, int64_t U1, int64_t T, int64_t N) {
+__host__ __device__ __forceinline__ int unit_contributors(int64_t U0, int64_t U1, int64_t T, int64_t N) {
     return T >= N ? (int)(cta_of(U1 - 1, T, N) - cta_of(U0, T, N) + 1) : (int)(U1 - U0);
+}
+
+// Partial slot of contributor j (in CTA order) of the unit starting at global
+// tile U0, whose first contributor is CTA c_first.  dense: T >= N (every CTA
+// range non-empty, contributors are consecutive CTAs); first_odd: the unit
+// starts inside c_first's range, so that CTA stored it as its second unit.
+// The writer of the partial uses partial_slot(); both must agree.
+__host__ __device__ __forceinline__ int64_t contributor_slot(int j, int64_t U0, int64_t c_first,
+                                                             bool first_odd, bool dense, int64_t T,
+                                                             int64_t N) {
+    const int64_t cc = dense ? c_first + j : cta_of(U0 + j, T, N);
+    return 2 * cc + ((j == 0 && first_odd) ? 1 : 0);
 }
 
 // Count one CTA's arrival at a split unit.  The CTA's partial stores are
@@ -195,8 +207,7 @@ __device__ __noinline__ void combine_partials(const Params& p, CombineSmem& cs, 
     // the first contributor's slot is odd when the unit starts inside its range
     const bool first_odd = range_start(c_first, T, N) < u.U0;
     auto part_of = [&](int j) -> const float* {
-        const int64_t cc = dense ? c_first + j : cta_of(u.U0 + j, T, N);
-        return p.partials + (2 * cc + ((j == 0 && first_odd) ? 1 : 0)) * slot_floats;
+        return p.partials + contributor_slot(j, u.U0, c_first, first_odd, dense, T, N) * slot_floats;
     };
     float4 acc[kOut4];
     float4 v[kOut4][kBatch];
