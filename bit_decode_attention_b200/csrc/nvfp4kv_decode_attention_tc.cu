@@ -861,7 +861,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
                         }
                 }
                 // arrival is counted after the roles finish, so that the
-                // fence and the atomic stay off this CTA's tile pipeline
+                // atomic (and the wait for its release) stays off this CTA's
+                // tile pipeline; a CTA splits at most its first and last unit
                 if (t == 0) sm.sig_gt[sm.n_sig++] = u.U0;
             }
             softmax_sync();
