@@ -6,6 +6,8 @@ import ctypes
 import glob
 import os
 import re
+import shutil
+import subprocess
 
 import pytest
 
@@ -151,3 +153,30 @@ def test_argument_validation_without_gpu(lib):
     assert cal(dev, 0, -1, dev, None, None) == INVALID
     assert cal(dev, 0, 10, None, None, None) == INVALID
     assert cal(ctypes.c_void_p(65), 0, 10, dev, None, None) == INVALID   # bf16 misaligned
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    # the boundary is a C ABI: a C99 program (-pedantic, no C++) includes the
+    # header, links the library and calls its host-only entry points
+    src = tmp_path / "abi.c"
+    src.write_text(
+        '#include "nvfp4kv.h"\n'
+        '#include <stdio.h>\n'
+        'int main(void) {\n'
+        '    nvfp4_kv_plane p = {0};\n'
+        '    nvfp4_kv_paged_plane q = {0};\n'
+        '    (void)p; (void)q;\n'
+        '    printf("%zu %zu %s\\n", nvfp4_cache_bytes(2, 8, 4096, 128), mxfp4_cache_bytes(2, 8, 4096, 128),\n'
+        '           nvfp4_status_string(NVFP4_ERR_CAPACITY));\n'
+        '    return 0;\n'
+        '}\n')
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(_native.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                    os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir, "-lnvfp4kv",
+                    "-Wl,-rpath," + libdir], check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert int(out[0]) == 2 * 8 * 4096 * (64 + 8)
+    assert int(out[1]) == 2 * 8 * 4096 * (64 + 4)
+    assert len(out) > 2
