@@ -2,15 +2,22 @@
 """NVFP4 KV-cache decode benchmark on B200: KV-tokens/s and achieved HBM GB/s.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload NAME] [--no-aux] [--no-cpu-baseline]
 
-One step is one pass of the whole decode hot path over one batch: quantize the
-new token's K and V (E2M1 codes + E4M3 block scales under the calibrated fp32
-tensor scale) and append them to the NVFP4 cache, then run decode attention
-over the cache with NVFP4 -> FP8 dequantization fused in.  Default workload:
-B=8 sequences, 32 query heads, 8 KV heads, head_dim 128, 4096 cached tokens +
-the appended one (4097 attended), bf16 inputs with per-channel log-normal
-scales.  Tensor-scale calibration and the 4096-token prefill quantization run
-once during set-up; their throughput is reported under "aux".
+One step is one pass of the whole decode hot path over one batch: quantize
+every sequence's new token (K and V: E2M1 codes + E4M3 block scales under the
+calibrated fp32 tensor scale) and append it to the NVFP4 cache, then run
+decode attention over the cache with the NVFP4 -> FP8 dequantization fused in
+(plus the merge of split units).
+
+Default workload ("ragged", the large-batch case): B=128 sequences, 32 query
+heads, 8 KV heads, head_dim 128, cached lengths uniform in [1024, 8192]
+(seeded) plus the appended token, contiguous per-sequence cache slabs, bf16
+inputs N(0,1) x per-channel LogNormal(0, 0.5).  Tensor-scale calibration and
+the prefill quantization run once during set-up; their throughput is reported
+under "aux", next to the other workloads' attention lines (64K context,
+128K context with GQA group 12 and 2048-token chunked appends, the 4K GQA
+decode step, a paged cache, a hot-L2 run).
 
 Timing: CUDA graphs of consecutive steps replayed on one stream, CUDA events
 around exactly K steps after W warm-up steps, barrier + synchronize on both
@@ -41,12 +48,15 @@ import synthetic  # noqa: E402
 
 METRIC = "NVFP4 decode-attention KV-tokens/s and achieved HBM GB/s (% of peak) at 1 B200"
 UNIT = "KV-tokens/s"
-DTYPE = "nvfp4 (e2m1 + e4m3 block scale) storage, fp8 e4m3 values, f16 MMA inputs, f32 accumulate"
+DTYPE = ("nvfp4 storage (e2m1 codes + e4m3 block scales + f32 tensor scale); e4m3 tcgen05 MMA "
+         "operands (K, V exact FP8; q as 2 e4m3 terms, P as 3 e4m3 terms); f32 accumulate")
+DEFAULT_WORKLOAD = "ragged"
 FALLBACK_HBM_GBS = 6650.0
 ATTN_SOURCES = ["bit_decode_attention_b200/csrc/nvfp4kv_decode_attention_tc.cu",
                 "bit_decode_attention_b200/csrc/nvfp4kv_attention_common.cuh",
                 "bit_decode_attention_b200/csrc/nvfp4kv_tcgen05.cuh",
                 "bit_decode_attention_b200/csrc/nvfp4kv_device.cuh"]
+GEN_SEQS = 16          # sequences drawn per host block when generating prefill inputs
 
 
 # ---------------------------------------------------------------------------
@@ -92,6 +102,27 @@ def profiled_traffic(name):
 def kv_bytes_per_token(Hkv, D):
     """Algorithmic HBM bytes to read one cached token (all KV heads, K and V)."""
     return Hkv * 2 * (D // 2 + D // 16)
+
+
+def gen_block(w, L, which, c):
+    """Host block c of the prefill inputs: sequences GEN_SEQS*c .. +GEN_SEQS-1,
+    fp32 values exact in the workload dtype, [nb][L][H_kv][D] (stream 1000 + c
+    of the workload's generator)."""
+    b0 = c * GEN_SEQS
+    nb = min(GEN_SEQS, w.B - b0)
+    return synthetic.kv_tokens(w, L, which, stream=1000 + c, batch=nb)
+
+
+def gen_inputs(w, L, which, device="cuda"):
+    """K or V prefill inputs [B][L][H_kv][D] in the workload dtype on `device`,
+    drawn on the host one block of GEN_SEQS sequences at a time (gen_block), so
+    host memory stays bounded."""
+    out = torch.empty(w.B, L, w.Hkv, w.D, dtype=w.torch_dtype(), device=device)
+    for c in range((w.B + GEN_SEQS - 1) // GEN_SEQS):
+        x = gen_block(w, L, which, c)
+        out[c * GEN_SEQS:c * GEN_SEQS + x.shape[0]].copy_(x.to(w.torch_dtype()))
+        del x
+    return out
 
 
 class ClockSampler:
@@ -162,83 +193,121 @@ class ClockSampler:
                 "samples": len(inside), "window": window}
 
 
+def time_events(fn, reps=5, warm=2):
+    """Average CUDA-event time (ms) of fn() over `reps` calls after `warm` calls."""
+    for _ in range(warm):
+        fn()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
 # ---------------------------------------------------------------------------
 # the decode workload
 # ---------------------------------------------------------------------------
 class DecodeWorkload:
-    """R replica NVFP4 caches of one workload, each prefilled with L0 tokens;
-    a step appends one token at slot L0 (the same slot every visit, so every
-    step attends exactly L0 + 1 tokens) and runs decode attention."""
+    """R replica NVFP4 caches of one workload.  Sequence b holds lens0[b]
+    cached tokens; a step appends one token at slot lens0[b] (the same slot
+    every visit, so every step attends exactly lens0[b] + 1 tokens) and runs
+    decode attention.  `prefill_chunk` prefills through appends of that many
+    tokens (timed); `measure_setup` times calibration, prefill, the MXFP4
+    codec and the standalone dequant on this workload."""
 
-    def __init__(self, w, L0, replicas, with_append=True, paged=False):
+    def __init__(self, w, replicas, with_append=True, paged=False, prefill_chunk=None,
+                 measure_setup=False):
         import bit_decode_attention_b200 as nv
         self.nv = nv
         assert not (paged and with_append), "the timed append writes contiguous planes"
-        self.w, self.L0, self.R, self.with_append, self.paged = w, L0, replicas, with_append, paged
+        self.w, self.R, self.with_append, self.paged = w, replicas, with_append, paged
         B, Hq, Hkv, D = w.B, w.Hq, w.Hkv, w.D
-        self.S_max = synthetic.capacity(L0 + 1)
+        self.lens0 = [int(x) for x in synthetic.seq_lens(w)]
+        L_max = max(self.lens0)
+        self.S_max = synthetic.capacity(L_max + 1)
         dev = "cuda"
-        bf = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-        xk = synthetic.kv_tokens(w, L0, "k")
-        xv = synthetic.kv_tokens(w, L0, "v")
+        dt = w.torch_dtype()
+        xk = gen_inputs(w, L_max, "k")
+        xv = gen_inputs(w, L_max, "v")
         nk = synthetic.kv_tokens(w, replicas, "k", stream=1)   # one new token per replica
         nv_ = synthetic.kv_tokens(w, replicas, "v", stream=1)
-        self.xk_d = xk.to(bf).to(dev)
-        self.xv_d = xv.to(bf).to(dev)
-        del xk, xv
-        self.new_k = [nk[:, j:j + 1].contiguous().to(bf).to(dev) for j in range(replicas)]
-        self.new_v = [nv_[:, j:j + 1].contiguous().to(bf).to(dev) for j in range(replicas)]
-        self.q = [synthetic.queries(w, stream=j).to(bf).to(dev) for j in range(replicas)]
+        self.new_k = [nk[:, j:j + 1].contiguous().to(dt).to(dev) for j in range(replicas)]
+        self.new_v = [nv_[:, j:j + 1].contiguous().to(dt).to(dev) for j in range(replicas)]
+        self.q = [synthetic.queries(w, stream=j).to(dt).to(dev) for j in range(replicas)]
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.aux = {}
         # calibration: one fp32 scale per tensor over every token the cache will hold
-        t0 = time.perf_counter()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        allk = torch.cat([self.xk_d, nk.to(bf).to(dev)], dim=1)
-        allv = torch.cat([self.xv_d, nv_.to(bf).to(dev)], dim=1)
-        ev[0].record()
+        allk = torch.cat([xk.reshape(-1), nk.to(dt).to(dev).reshape(-1)])
+        allv = torch.cat([xv.reshape(-1), nv_.to(dt).to(dev).reshape(-1)])
         self.sk = nv.nvfp4_calib_tensor_scale(allk, status=self.status)
         self.sv = nv.nvfp4_calib_tensor_scale(allv, status=self.status)
-        ev[1].record()
-        torch.cuda.synchronize()
-        self.calib_ms = ev[0].elapsed_time(ev[1])
-        self.calib_bytes = (allk.numel() + allv.numel()) * allk.element_size()
+        if measure_setup:
+            ms = time_events(lambda: (nv.nvfp4_calib_tensor_scale(allk, self.sk, status=self.status),
+                                      nv.nvfp4_calib_tensor_scale(allv, self.sv, status=self.status)))
+            nbytes = (allk.numel() + allv.numel()) * allk.element_size()
+            self.aux["calib_gbs"] = nbytes / (ms / 1e3) / 1e9
+            self.aux["calib_note"] = ("warm, mean of 5 calls; K and V calibrated over %.0f MB of %s"
+                                      % (nbytes / 1e6, w.dtype))
         del allk, allv
-        # replica caches, prefilled
-        self.k, self.v, self.out = [], [], []
+        # replica 0 prefilled through the quantizer, the others copied from it
         zeros = torch.zeros(B, dtype=torch.int32, device=dev)
-        self.prefill_ms = 0.0
-        for r in range(replicas):
-            k = nv.KVPlane.allocate(B, Hkv, self.S_max, D)
-            v = nv.KVPlane.allocate(B, Hkv, self.S_max, D)
-            ev[0].record()
-            nv.nvfp4_kv_quantize_append(self.xk_d, zeros, self.sk, k, status=self.status)
-            nv.nvfp4_kv_quantize_append(self.xv_d, zeros, self.sv, v, status=self.status)
-            ev[1].record()
-            torch.cuda.synchronize()
-            self.prefill_ms += ev[0].elapsed_time(ev[1])
+        k0 = nv.KVPlane.allocate(B, Hkv, self.S_max, D)
+        v0 = nv.KVPlane.allocate(B, Hkv, self.S_max, D)
+        elems = 2 * B * L_max * Hkv * D
+        if prefill_chunk:
+            starts = [torch.full((B,), lo, dtype=torch.int32, device=dev)
+                      for lo in range(0, L_max, prefill_chunk)]
+            chunks = [(xk[:, lo:lo + prefill_chunk].contiguous(), xv[:, lo:lo + prefill_chunk].contiguous())
+                      for lo in range(0, L_max, prefill_chunk)]
+
+            def prefill():
+                for s, (a, b) in zip(starts, chunks):
+                    nv.nvfp4_kv_quantize_append_kv(a, b, s, self.sk, self.sv, k0, v0, status=self.status)
+            ms = time_events(prefill, reps=3, warm=1)
+            self.aux["chunked_append_gbs"] = (elems * xk.element_size() + elems * 9 // 16) / (ms / 1e3) / 1e9
+            self.aux["chunked_append_note"] = ("%d appends of %d tokens x B%d x %d KV heads, K and V per launch, "
+                                               "mean of 3 passes" % (len(starts), prefill_chunk, B, Hkv))
+            del chunks
+        else:
+            def prefill():
+                nv.nvfp4_kv_quantize_append_kv(xk, xv, zeros, self.sk, self.sv, k0, v0, status=self.status)
+            if measure_setup:
+                ms = time_events(prefill, reps=3, warm=1)
+                self.aux["prefill_quantize_gbs"] = (elems * xk.element_size() + elems * 9 // 16) / (ms / 1e3) / 1e9
+            else:
+                prefill()
+        if measure_setup:
+            # the MXFP4 comparison codec on the same prefill (32-element blocks,
+            # E8M0 scales): 0.53125 B written per element
+            mk = nv.KVPlane.allocate_mxfp4(B, Hkv, self.S_max, D)
+            mv = nv.KVPlane.allocate_mxfp4(B, Hkv, self.S_max, D)
+            ms = time_events(lambda: (nv.mxfp4_kv_quantize_append(xk, zeros, mk, status=self.status),
+                                      nv.mxfp4_kv_quantize_append(xv, zeros, mv, status=self.status)),
+                             reps=3, warm=1)
+            self.aux["mxfp4_prefill_quantize_gbs"] = (elems * xk.element_size() + elems * 17 // 32) / (ms / 1e3) / 1e9
+            del mk, mv
+            # the standalone dequant to FP8 (0.5625 B read + 1 B written per element)
+            lens_t = torch.tensor(self.lens0, dtype=torch.int32, device=dev)
+            fp8 = torch.empty(B, Hkv, self.S_max, D, dtype=torch.uint8, device=dev)
+            ms = time_events(lambda: nv.nvfp4_kv_dequant_fp8(k0, self.sk, lens_t, out=fp8, status=self.status))
+            self.aux["dequant_fp8_gbs"] = sum(self.lens0) * Hkv * D * (1 + 9 / 16) / (ms / 1e3) / 1e9
+            del fp8
+        del xk, xv
+        self.k, self.v, self.out = [k0], [v0], []
+        for r in range(1, replicas):
+            k = nv.KVPlane(k0.codes.clone(), k0.scales.clone())
+            v = nv.KVPlane(v0.codes.clone(), v0.scales.clone())
             self.k.append(k)
             self.v.append(v)
+        for r in range(replicas):
             self.out.append(torch.empty(B, Hq, D, dtype=torch.float32, device=dev))
-        elems = 2 * B * L0 * Hkv * D
-        self.prefill_bytes = replicas * (elems * self.xk_d.element_size() + elems * 9 // 16)
-        # the MXFP4 comparison codec on the same prefill (32-element blocks, E8M0
-        # scales): 0.53125 B written per element; timed, then freed
-        mk = nv.KVPlane.allocate_mxfp4(B, Hkv, self.S_max, D)
-        mv = nv.KVPlane.allocate_mxfp4(B, Hkv, self.S_max, D)
-        reps = 3
-        ev[0].record()
-        for _ in range(reps):
-            nv.mxfp4_kv_quantize_append(self.xk_d, zeros, mk, status=self.status)
-            nv.mxfp4_kv_quantize_append(self.xv_d, zeros, mv, status=self.status)
-        ev[1].record()
-        torch.cuda.synchronize()
-        self.mx_prefill_ms = ev[0].elapsed_time(ev[1]) / reps
-        self.mx_prefill_bytes = elems * self.xk_d.element_size() + elems * 17 // 32
-        del mk, mv
-        self.start = torch.full((B,), L0, dtype=torch.int32, device=dev)
-        self.lens = torch.full((B,), L0 + 1 if with_append else L0, dtype=torch.int32, device=dev)
+        self.start = torch.tensor(self.lens0, dtype=torch.int32, device=dev)
+        self.lens_att = [L + 1 for L in self.lens0] if with_append else list(self.lens0)
+        self.lens = torch.tensor(self.lens_att, dtype=torch.int32, device=dev)
         self.ws = nv.new_workspace(B, Hq, Hkv, D)
-        self.L_att = L0 + 1 if with_append else L0
         if paged:
             self._page_replicas(nv)
         torch.cuda.synchronize()
@@ -264,32 +333,37 @@ class DecodeWorkload:
                 planes.append(nv.PagedKVPlane(pools[0], pools[1], table))
             self.k[r], self.v[r] = planes
 
-    # kernels per step (ours): 1 append of K and V + 1 attention
+    # kernels per step (ours): the attention kernel (which appends the new
+    # tokens itself on the tensor-core path) + the split-K merge
     @property
     def launches_per_step(self):
-        return 2 if self.with_append else 1
+        return 2
 
     def tokens_per_step(self):
-        return self.w.B * self.L_att
+        return sum(self.lens_att)
 
     def attention_bytes(self):
         """Algorithmic bytes of one attention launch: cache reads + q + out."""
         w = self.w
-        kv = self.w.B * self.L_att * kv_bytes_per_token(w.Hkv, w.D)
+        kv = self.tokens_per_step() * kv_bytes_per_token(w.Hkv, w.D)
         qb = w.B * w.Hq * w.D * self.q[0].element_size()
         ob = w.B * w.Hq * w.D * 4
         return kv + qb + ob
 
     def step(self, j, events=None):
+        """One decode step on replica j % R: append + attention in one call
+        (nvfp4_decode_attention_append), or attention alone."""
         nv, r = self.nv, j % self.R
-        if self.with_append:
-            nv.nvfp4_kv_quantize_append_kv(self.new_k[r], self.new_v[r], self.start, self.sk, self.sv,
-                                           self.k[r], self.v[r], status=self.status)
         if events is not None:
             events[0].record()
-        attend = nv.nvfp4_decode_attention_paged if self.paged else nv.nvfp4_decode_attention
-        attend(self.q[r], self.k[r], self.v[r], self.sk, self.sv, self.lens,
-               out=self.out[r], workspace=self.ws, status=self.status)
+        if self.with_append:
+            nv.nvfp4_decode_attention_append(self.q[r], self.new_k[r], self.new_v[r], self.start, self.k[r],
+                                             self.v[r], self.sk, self.sv, out=self.out[r], workspace=self.ws,
+                                             status=self.status)
+        else:
+            attend = nv.nvfp4_decode_attention_paged if self.paged else nv.nvfp4_decode_attention
+            attend(self.q[r], self.k[r], self.v[r], self.sk, self.sv, self.lens,
+                   out=self.out[r], workspace=self.ws, status=self.status)
         if events is not None:
             events[1].record()
 
@@ -322,7 +396,7 @@ def run_steps(graph_full, graph_tail, per_graph, n_steps):
 
 
 def time_decode(wl, steps, warmup, world, sampler=None, graph_steps=None, nvtx_name="timed"):
-    """Returns (elapsed_ms max over ranks, attention ms per launch, clocks)."""
+    """Returns (elapsed_ms max over ranks, attention ms per launch, launches sampled, clocks)."""
     G = graph_steps or wl.R * max(1, 16 // wl.R)
     G = max(G, wl.R)
     G -= G % wl.R
@@ -354,9 +428,10 @@ def time_decode(wl, steps, warmup, world, sampler=None, graph_steps=None, nvtx_n
 
 
 def time_e2e(wl, steps):
-    """Same step through the public API from pinned host buffers: per step
-    H2D of the new K/V token and the query, the step's launches, D2H of the
-    attention output.  Returns (ms, h2d bytes/step, d2h bytes/step)."""
+    """The same step through the public API from pinned host buffers: per step
+    H2D of the new K/V token (when the step appends) and the query, the step's
+    launches, D2H of the attention output.  Returns (ms, h2d bytes/step, d2h
+    bytes/step)."""
     nv = wl.nv
     R = wl.R
     h_k = [t.cpu().pin_memory() for t in wl.new_k]
@@ -366,16 +441,20 @@ def time_e2e(wl, steps):
     d_k = [torch.empty_like(t) for t in wl.new_k]
     d_v = [torch.empty_like(t) for t in wl.new_v]
     d_q = [torch.empty_like(t) for t in wl.q]
+    attend = nv.nvfp4_decode_attention_paged if wl.paged else nv.nvfp4_decode_attention
 
     def one(j):
         r = j % R
-        d_k[r].copy_(h_k[r], non_blocking=True)
-        d_v[r].copy_(h_v[r], non_blocking=True)
+        if wl.with_append:
+            d_k[r].copy_(h_k[r], non_blocking=True)
+            d_v[r].copy_(h_v[r], non_blocking=True)
         d_q[r].copy_(h_q[r], non_blocking=True)
-        nv.nvfp4_kv_quantize_append_kv(d_k[r], d_v[r], wl.start, wl.sk, wl.sv, wl.k[r], wl.v[r],
-                                       status=wl.status)
-        nv.nvfp4_decode_attention(d_q[r], wl.k[r], wl.v[r], wl.sk, wl.sv, wl.lens, out=wl.out[r],
-                                  workspace=wl.ws, status=wl.status)
+        if wl.with_append:
+            nv.nvfp4_decode_attention_append(d_q[r], d_k[r], d_v[r], wl.start, wl.k[r], wl.v[r], wl.sk, wl.sv,
+                                             out=wl.out[r], workspace=wl.ws, status=wl.status)
+        else:
+            attend(d_q[r], wl.k[r], wl.v[r], wl.sk, wl.sv, wl.lens, out=wl.out[r], workspace=wl.ws,
+                   status=wl.status)
         h_out[r].copy_(wl.out[r], non_blocking=True)
 
     for j in range(min(steps, 3 * R)):
@@ -387,28 +466,60 @@ def time_e2e(wl, steps):
         one(j)
     b.record()
     torch.cuda.synchronize()
-    h2d = (d_k[0].numel() * d_k[0].element_size() + d_v[0].numel() * d_v[0].element_size()
-           + d_q[0].numel() * d_q[0].element_size())
+    h2d = d_q[0].numel() * d_q[0].element_size()
+    if wl.with_append:
+        h2d += d_k[0].numel() * d_k[0].element_size() + d_v[0].numel() * d_v[0].element_size()
     d2h = wl.out[0].numel() * 4
     return a.elapsed_time(b), h2d, d2h
+
+
+def roofline_block(wl, att_ms, att_n, peak, peak_kind, traffic_name=None):
+    """HBM roofline of the step's attention call (append + attention when the
+    step appends): algorithmic cache bytes / event-timed call duration."""
+    if not att_ms:
+        return None
+    achieved = wl.attention_bytes() / (att_ms / 1e3) / 1e9
+    g = wl.w.Hq // wl.w.Hkv
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak,
+            "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+            else "fallback",
+            "traffic": profiled_traffic(traffic_name) if traffic_name else None,
+            "kernel": "decode_attention_tc_kernel<%d> + merge_split_units_kernel (tcgen05, head_dim "
+                      "128, bf16 queries, GQA group %d)" % (1 if g <= 8 else 2, g),
+            "algorithmic_bytes_per_launch": wl.attention_bytes(),
+            "launch_ms": att_ms, "launches_sampled": att_n,
+            "frac_of_nominal_8tbs": achieved / 8000.0}
+
+
+def workload_label(w, wl):
+    lens = "L %d" % w.L if w.L is not None else "L~U[%d,%d] (sum %d)" % (
+        w.L_range[0], w.L_range[1], sum(wl.lens0))
+    what = ("append 1 token per sequence (K and V) + decode attention" if wl.with_append
+            else "decode attention")
+    return "%s: B%d Hq%d Hkv%d D%d, %s cached tokens, %s%s" % (
+        w.name, w.B, w.Hq, w.Hkv, w.D, lens, what, " over 128-token pages" if wl.paged else "")
 
 
 # ---------------------------------------------------------------------------
 # CPU oracle timings (cpu_baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
 class OracleSample:
-    """The oracle's decode step for ONE sequence of the workload: quantize and
-    append its new K/V token, then fp64 decode attention over L0 + 1 tokens.
-    Inputs are the same seeded tensors the GPU run uses."""
+    """The oracle's decode step for ONE sequence of the workload (with sequence
+    0's length): quantize and append its new K/V token, then fp64 decode
+    attention over its cached tokens + 1.  Inputs come from the same seeded
+    distributions as the GPU run's."""
 
-    def __init__(self, w, L0, seconds_hint=None):
+    def __init__(self, w, L0=None):
         import oracle
         self.oracle = oracle
-        self.w, self.L0 = w, L0
+        self.w = w
+        L0 = L0 if L0 is not None else int(synthetic.seq_lens(w)[0])
+        self.L0 = L0
         S_max = synthetic.capacity(L0 + 1)
         one = synthetic.shrink(w, B=1)
-        xk = synthetic.kv_tokens(one, L0, "k")
-        xv = synthetic.kv_tokens(one, L0, "v")
+        xk = synthetic.kv_tokens(one, L0, "k", stream=1000)
+        xv = synthetic.kv_tokens(one, L0, "v", stream=1000)
         self.nk = synthetic.kv_tokens(one, 1, "k", stream=1).numpy()
         self.nv = synthetic.kv_tokens(one, 1, "v", stream=1).numpy()
         self.q = synthetic.queries(one).numpy()
@@ -434,14 +545,14 @@ class OracleSample:
         return self.L0 + 1
 
 
-def cpu_baseline(w, L0, budget_s=15.0, single_budget_s=5.0):
+def cpu_baseline(w, budget_s=15.0, single_budget_s=5.0):
     """The oracle, untuned, on every host core (OpenMP over KV heads), and
     single-threaded on a shorter budget."""
     import oracle
 
     def timed(threads, budget):
         oracle.set_threads(threads)
-        s = OracleSample(w, L0)
+        s = OracleSample(w)
         s.step()
         n, t0 = 0, time.perf_counter()
         while True:
@@ -455,19 +566,19 @@ def cpu_baseline(w, L0, budget_s=15.0, single_budget_s=5.0):
     n1, tok1, dt1, _ = timed(1, single_budget_s)
     n, tok, dt, cores = timed(os.cpu_count() or 1, budget_s)
     return {"value": n * tok / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": "%d oracle decode steps of one sequence (append 1 token + fp64 attention over "
-                      "%d tokens, %d KV heads, group %d) in %.1f s" % (n, tok, w.Hkv, w.g, dt),
+            "sample": "%d oracle decode steps of one sequence of the workload (append 1 token + fp64 "
+                      "attention over %d tokens, %d KV heads, group %d) in %.1f s" % (n, tok, w.Hkv, w.g, dt),
             "single_thread": {"value": n1 * tok1 / dt1, "unit": UNIT, "cores": 1,
                               "sample": "%d steps in %.1f s" % (n1, dt1)}}
 
 
-def run_reference(args, rank, world, w, L0):
+def run_reference(args, rank, world, w):
     if rank != 0:
         return
     import oracle
     threads = os.cpu_count() or 1
     oracle.set_threads(threads)
-    s = OracleSample(w, L0)
+    s = OracleSample(w)
     # size the per-step sample so warm-up + steps end in about two minutes:
     # every KV head of one sequence, over a prefix of L_s cached tokens
     t0 = time.perf_counter()
@@ -475,6 +586,7 @@ def run_reference(args, rank, world, w, L0):
     full = time.perf_counter() - t0
     total = args.steps + args.warmup
     per_step_budget = 120.0 / max(total, 1)
+    L0 = s.L0
     L_s = L0 if full <= per_step_budget else max(16, int(L0 * per_step_budget / full))
     sub = s if L_s == L0 else OracleSample(w, L_s)
     for _ in range(args.warmup):
@@ -485,13 +597,13 @@ def run_reference(args, rank, world, w, L0):
     dt = time.perf_counter() - t0
     tokens = args.steps * sub.tokens
     value = tokens / dt
-    desc = ("per step: oracle append + fp64 decode attention for 1 sequence, all %d KV heads, "
-            "%d tokens (of %d)" % (w.Hkv, sub.tokens, L0 + 1))
+    desc = ("per step: oracle append + fp64 decode attention for 1 sequence of the workload, all %d KV "
+            "heads, %d tokens (of %d)" % (w.Hkv, sub.tokens, L0 + 1))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(args.steps, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
-        "data": "synthetic (seeded)", "config": config_block(w, L0, None),
+        "data": "synthetic (seeded)", "config": config_block(w, None),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.get_threads(), "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -499,10 +611,15 @@ def run_reference(args, rank, world, w, L0):
     print(json.dumps(line), flush=True)
 
 
-def config_block(w, L0, wl):
-    cfg = {"workload": "%s: B%d Hq%d Hkv%d D%d, %d cached + 1 appended token per step, append K/V "
-                       "+ decode attention" % (w.name, w.B, w.Hq, w.Hkv, w.D, L0),
-           "B": w.B, "H_q": w.Hq, "H_kv": w.Hkv, "head_dim": w.D, "seq_len": L0 + 1,
+def config_block(w, wl):
+    lens = [int(x) for x in synthetic.seq_lens(w)]
+    cfg = {"workload": "%s: B%d Hq%d Hkv%d D%d, %s cached tokens + 1 appended per sequence per step, "
+                       "append K/V + decode attention" % (
+                           w.name, w.B, w.Hq, w.Hkv, w.D,
+                           ("L %d" % w.L) if w.L is not None else
+                           ("L~U[%d,%d] seeded, sum %d" % (w.L_range[0], w.L_range[1], sum(lens)))),
+           "B": w.B, "H_q": w.Hq, "H_kv": w.Hkv, "head_dim": w.D,
+           "seq_len": (w.L + 1) if w.L is not None else [min(lens) + 1, max(lens) + 1],
            "input_dtype": w.dtype, "parallelism": "replicas"}
     if wl is not None:
         touched = wl.R * wl.attention_bytes()
@@ -530,25 +647,52 @@ def replicas_for(bytes_per_replica, l2_bytes):
     return max(2, math.ceil(2 * l2_bytes / bytes_per_replica))
 
 
+def aux_attention(name, w, l2, steps, world, peak, peak_kind, with_append=False, paged=False,
+                  replicas=None, prefill_chunk=None, e2e_steps=200, label_extra=""):
+    """Timed aux line for one workload: attention (or the append + attention
+    step), its roofline, and the same through the public API from host buffers."""
+    lens = synthetic.seq_lens(w)
+    per = (sum(lens) + len(lens)) * kv_bytes_per_token(w.Hkv, w.D)
+    R = replicas or replicas_for(per, l2)
+    wl = DecodeWorkload(w, R, with_append=with_append, paged=paged, prefill_chunk=prefill_chunk)
+    ms, att, att_n, _ = time_decode(wl, steps, 20, world, nvtx_name="timed_aux_" + name)
+    e2e_ms, h2d, d2h = time_e2e(wl, e2e_steps)
+    tok = wl.tokens_per_step()
+    roof = roofline_block(wl, att, att_n, peak, peak_kind, "decode_attention_%s_traffic.json" % name)
+    line = {"workload": workload_label(w, wl) + label_extra,
+            "kv_tokens_per_s": world * tok * steps / (ms / 1e3), "ms_per_step": ms / steps,
+            "steps": steps, "replicas": R, "roofline": roof,
+            "launch_ms": att, "achieved_gbs": roof["achieved"] if roof else None,
+            "frac_of_measured": roof["frac"] if roof else None,
+            "e2e": {"value": world * tok * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}}
+    line.update(wl.aux)
+    status = wl.status.item()
+    if status:
+        line["device_status"] = status
+    del wl
+    torch.cuda.empty_cache()
+    return line
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", default="gqa", choices=[w.name for w in synthetic.WORKLOADS])
-    ap.add_argument("--no-aux", action="store_true", help="skip the 64K attention-only line")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=[w.name for w in synthetic.WORKLOADS])
+    ap.add_argument("--no-aux", action="store_true", help="skip the other workloads' lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--e2e-steps", type=int, default=500)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     rank, world, local_rank = env_rank()
     w = synthetic.get(args.workload)
-    L0 = w.L if w.L is not None else w.L_range[1]
 
     if args.impl == "reference":
-        run_reference(args, rank, world, w, L0)
+        run_reference(args, rank, world, w)
         return
 
     torch.cuda.set_device(local_rank)
@@ -557,39 +701,29 @@ def main():
                                              device_id=torch.device("cuda", local_rank))
     props = torch.cuda.get_device_properties(local_rank)
     l2 = getattr(props, "L2_cache_size", 126 * 1024 * 1024)
-    per_replica = w.B * (L0 + 1) * kv_bytes_per_token(w.Hkv, w.D)
+    lens = synthetic.seq_lens(w)
+    per_replica = (sum(lens) + len(lens)) * kv_bytes_per_token(w.Hkv, w.D)
     R = replicas_for(per_replica, l2)
-    wl = DecodeWorkload(w, L0, R)
+    wl = DecodeWorkload(w, R, measure_setup=True)
     sampler = ClockSampler(local_rank)
     sampler.start()
     time.sleep(0.3)
     ms, att_ms, att_n, clocks = time_decode(wl, args.steps, args.warmup, world, sampler)
     sampler.stop()
-    e2e_ms, h2d, d2h = time_e2e(wl, min(args.e2e_steps, args.steps))
     e2e_steps = min(args.e2e_steps, args.steps)
+    e2e_ms, h2d, d2h = time_e2e(wl, e2e_steps)
     status = wl.status.item()
 
     tokens = wl.tokens_per_step()
     value = job_throughput(world, tokens, args.steps, ms)
     peak, peak_kind = measured_peaks()
-    roof = None
-    if att_ms:
-        achieved = wl.attention_bytes() / (att_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)"
-                if peak_kind == "measured" else "fallback",
-                "traffic": profiled_traffic("decode_attention_%s_traffic.json" % w.name),
-                "kernel": "decode_attention_tc_kernel<%d> (tcgen05, head_dim 128, bf16 queries)"
-                          % (1 if w.Hq // w.Hkv <= 8 else 2),
-                "algorithmic_bytes_per_launch": wl.attention_bytes(),
-                "launch_ms": att_ms, "launches_sampled": att_n,
-                "frac_of_nominal_8tbs": achieved / 8000.0}
+    roof = roofline_block(wl, att_ms, att_n, peak, peak_kind, "decode_attention_%s_traffic.json" % w.name)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": DTYPE,
         "data": "synthetic (seeded; bf16 K/V ~ N(0,1) x per-channel LogNormal, no weights needed)",
-        "config": config_block(w, L0, wl),
+        "config": config_block(w, wl),
         "hbm_gbs_step": world * tokens * kv_bytes_per_token(w.Hkv, w.D) * args.steps / (ms / 1e3) / 1e9,
         "roofline": roof,
         "e2e": {"value": world * tokens * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
@@ -599,42 +733,25 @@ def main():
         "clocks": clocks,
         "device_status": status,
     }
-    aux = {"calib_gbs": wl.calib_bytes / (wl.calib_ms / 1e3) / 1e9,
-           "prefill_quantize_gbs": wl.prefill_bytes / (wl.prefill_ms / 1e3) / 1e9,
-           "mxfp4_prefill_quantize_gbs": wl.mx_prefill_bytes / (wl.mx_prefill_ms / 1e3) / 1e9}
+    aux = dict(wl.aux)
     del wl
     torch.cuda.empty_cache()
     if not args.no_aux:
-        lw = synthetic.get("long64k")
-        per = lw.B * lw.L * kv_bytes_per_token(lw.Hkv, lw.D)
-        lwl = DecodeWorkload(lw, lw.L, replicas_for(per, l2), with_append=False)
         n_aux = max(64, min(2000, args.steps))
-        lms, latt, lat_n, _ = time_decode(lwl, n_aux, 20, world, nvtx_name="timed_aux")
-        ach = lwl.attention_bytes() / (latt / 1e3) / 1e9 if latt else None
-        aux["long64k_attention"] = {
-            "workload": "long64k: B1 Hq64 Hkv8 D128 L65536, decode attention only (split-K)",
-            "kv_tokens_per_s": world * lwl.tokens_per_step() * n_aux / (lms / 1e3),
-            "launch_ms": latt, "achieved_gbs": ach, "frac_of_measured": ach / peak if ach else None,
-            "frac_of_nominal_8tbs": ach / 8000.0 if ach else None, "steps": n_aux,
-            "replicas": lwl.R}
-        del lwl
-        torch.cuda.empty_cache()
-        # the gqa attention over a paged cache (128-token pages, shuffled block table)
-        gw = synthetic.get("gqa")
-        per = gw.B * gw.L * kv_bytes_per_token(gw.Hkv, gw.D)
-        pwl = DecodeWorkload(gw, gw.L, replicas_for(per, l2), with_append=False, paged=True)
-        pms, patt, pat_n, _ = time_decode(pwl, n_aux, 20, world, nvtx_name="timed_aux_paged")
-        pach = pwl.attention_bytes() / (patt / 1e3) / 1e9 if patt else None
-        aux["gqa_paged_attention"] = {
-            "workload": "gqa paged: B8 Hq32 Hkv8 D128 L4096, 128-token pages in shuffled order",
-            "kv_tokens_per_s": world * pwl.tokens_per_step() * n_aux / (pms / 1e3),
-            "launch_ms": patt, "achieved_gbs": pach, "frac_of_measured": pach / peak if pach else None,
-            "steps": n_aux, "replicas": pwl.R}
-        del pwl
-        torch.cuda.empty_cache()
+        aux["long64k_attention"] = aux_attention("long64k", synthetic.get("long64k"), l2, n_aux, world,
+                                                 peak, peak_kind)
+        aux["moe128k_attention"] = aux_attention("moe128k", synthetic.get("moe128k"), l2, n_aux, world,
+                                                 peak, peak_kind, prefill_chunk=2048)
+        aux["gqa_step"] = aux_attention("gqa", synthetic.get("gqa"), l2, n_aux, world, peak, peak_kind,
+                                        with_append=True)
+        aux["gqa_paged_attention"] = aux_attention("gqa_paged", synthetic.get("gqa"), l2, n_aux, world,
+                                                   peak, peak_kind, paged=True)
+        aux["gqa_attention_hot_l2"] = aux_attention(
+            "gqa_hot", synthetic.get("gqa"), l2, n_aux, world, peak, peak_kind, replicas=1,
+            label_extra=" -- HOT L2: one cache (38 MB < L2) re-read every step, not a DRAM number")
     line["aux"] = aux
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, L0)
+        line["cpu_baseline"] = cpu_baseline(w)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

@@ -120,6 +120,12 @@ def nvfp4_version() -> str:
     return _native.lib().nvfp4_version().decode()
 
 
+def nvfp4_set_wait_limit(polls: int) -> None:
+    """Testing hook: pipeline-wait give-up limit of the tensor-core attention
+    kernel (sleeping polls; 0 = give up unless already complete; < 0 = default)."""
+    _native.lib().nvfp4_set_wait_limit(int(polls))
+
+
 def nvfp4_cache_bytes(B: int, H_kv: int, S_max: int, D: int) -> int:
     return int(_native.lib().nvfp4_cache_bytes(B, H_kv, S_max, D))
 
@@ -244,6 +250,35 @@ def nvfp4_decode_attention(q: torch.Tensor, k: KVPlane, v: KVPlane, s_tensor_k: 
         _ptr(s_tensor_v), _ptr(seq_lens), ctypes.c_float(softmax_scale), _ptr(out),
         _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
     _native.check("nvfp4_decode_attention", st)
+    return out
+
+
+def nvfp4_decode_attention_append(q: torch.Tensor, x_k_new: torch.Tensor, x_v_new: torch.Tensor,
+                                  start_pos: torch.Tensor, k: KVPlane, v: KVPlane, s_tensor_k: torch.Tensor,
+                                  s_tensor_v: torch.Tensor, softmax_scale: float = 0.0,
+                                  out: Optional[torch.Tensor] = None, new_lens: Optional[torch.Tensor] = None,
+                                  workspace: Optional[torch.Tensor] = None,
+                                  status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Append one token per sequence (x_k_new / x_v_new [B][1][H_kv][D]) at slot
+    start_pos[b], then attend over start_pos[b] + 1 tokens; fp32 [B][H_q][D]."""
+    _need_cuda(q, x_k_new, x_v_new, start_pos, s_tensor_k, s_tensor_v, out, new_lens, workspace, status)
+    if x_k_new.shape != x_v_new.shape or x_k_new.dtype != x_v_new.dtype:
+        raise ValueError("x_k_new and x_v_new must have the same shape and dtype")
+    B, H_q, D = q.shape
+    Bk, H_kv, S, Dk = k.shape
+    if tuple(x_k_new.shape) != (Bk, 1, H_kv, Dk):
+        raise ValueError("x_k_new must be [B][1][H_kv][D]")
+    if out is None:
+        out = torch.empty(B, H_q, D, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(B, H_q, H_kv, D, device=q.device)
+    kp, vp = k.struct(), v.struct()
+    st = _native.lib().nvfp4_decode_attention_append(
+        _ptr(q), _dtype_code(q), H_q, _ptr(x_k_new), _ptr(x_v_new), _dtype_code(x_k_new), _ptr(start_pos),
+        _ptr(new_lens), ctypes.byref(kp), ctypes.byref(vp), _ptr(s_tensor_k), _ptr(s_tensor_v),
+        ctypes.c_float(softmax_scale), _ptr(out), _ptr(workspace), workspace.numel(), _ptr(status),
+        _stream(stream))
+    _native.check("nvfp4_decode_attention_append", st)
     return out
 
 

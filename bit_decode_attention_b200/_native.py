@@ -38,6 +38,8 @@ EXPORTS = (
     "mxfp4_kv_quantize_append",
     "nvfp4_kv_quantize_append_paged",
     "nvfp4_decode_attention_paged",
+    "nvfp4_decode_attention_append",
+    "nvfp4_set_wait_limit",
 )
 
 
@@ -120,6 +122,11 @@ def lib():
     L.nvfp4_decode_attention_paged.argtypes = [vp, i32, i32, paged_p, paged_p, vp, vp, vp, f32, vp, vp,
                                                sz, vp, vp]
     L.nvfp4_decode_attention_paged.restype = i32
+    L.nvfp4_decode_attention_append.argtypes = [vp, i32, i32, vp, vp, i32, vp, vp, plane_p, plane_p, vp, vp,
+                                                f32, vp, vp, sz, vp, vp]
+    L.nvfp4_decode_attention_append.restype = i32
+    L.nvfp4_set_wait_limit.argtypes = [i64]
+    L.nvfp4_set_wait_limit.restype = None
     _lib = L
     return L
 

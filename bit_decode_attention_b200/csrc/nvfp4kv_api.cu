@@ -4,6 +4,8 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
+#include <mutex>
 
 #include <cuda_runtime.h>
 
@@ -12,19 +14,41 @@
 
 namespace nvfp4kv {
 
+namespace {
+std::mutex g_dev_mutex;
+int g_sm_count[kMaxDevices] = {};   // 0 = not looked up yet
+}  // namespace
+
 int device_sm_count() {
-    static int cached_dev = -1;
-    static int cached_count = 0;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-    if (dev != cached_dev) {
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev >= kMaxDevices) {
+        int n = 0;
+        return (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) ? n : 148;
+    }
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (g_sm_count[dev] == 0) {
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
             n = 148;
-        cached_count = n;
-        cached_dev = dev;
+        g_sm_count[dev] = n;
     }
-    return cached_count;
+    return g_sm_count[dev];
+}
+
+cudaError_t ensure_smem_attribute(const void* kernel, int bytes, int* done_flags) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices)
+        return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!done_flags[dev]) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e != cudaSuccess) return e;
+        done_flags[dev] = 1;
+    }
+    return cudaSuccess;
 }
 
 AttnWorkspace attention_workspace(int B, int Hq, int Hkv, int D) {
@@ -42,6 +66,12 @@ AttnWorkspace attention_workspace(int B, int Hq, int Hkv, int D) {
 namespace {
 
 using namespace nvfp4kv;
+
+// Give-up limit of the tensor-core attention kernel's pipeline waits, in
+// sleeping polls of up to 20 us each (2^16: about a second or more);
+// nvfp4_set_wait_limit changes it (a testing hook).
+constexpr uint32_t kDefaultWaitPolls = 1u << 16;
+std::atomic<uint32_t> g_wait_polls{kDefaultWaitPolls};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -77,11 +107,12 @@ struct CacheView {
 
 // Validation and batch-chunked launches shared by the contiguous and the
 // paged attention entry points (the planes are already validated).
-nvfp4_status run_attention(const void* q, nvfp4_dtype q_dtype, int H_q, int B, int H_kv, int D,
-                           int S_max, const CacheView& c, const float* d_s_tensor_k,
-                           const float* d_s_tensor_v, const int32_t* d_seq_lens, float softmax_scale,
-                           float* out, void* workspace, size_t workspace_bytes, int32_t* d_status,
-                           nvfp4_stream_t stream) {
+// Argument checks shared by every attention entry point (the planes are
+// already validated): dtype, group size, pointers, alignment, softmax scale,
+// and the 32-bit tile count of one launch.
+nvfp4_status check_attention_args(const void* q, nvfp4_dtype q_dtype, int H_q, int B, int H_kv, int S_max,
+                                  const float* d_s_tensor_k, const float* d_s_tensor_v,
+                                  const int32_t* d_seq_lens, float softmax_scale, const float* out) {
     if (q_dtype != NVFP4_IN_BF16 && q_dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
     if (H_q <= 0 || (H_q % H_kv) != 0) return NVFP4_ERR_INVALID_ARG;
     if (H_q / H_kv > 16) return NVFP4_ERR_UNSUPPORTED;
@@ -95,6 +126,26 @@ nvfp4_status run_attention(const void* q, nvfp4_dtype q_dtype, int H_q, int B, i
     const int64_t launch_tiles = (int64_t)(B < kMaxBatchPerLaunch ? B : kMaxBatchPerLaunch) * H_kv *
                                  (((int64_t)S_max + 31) / 32);
     if (launch_tiles > (int64_t)INT32_MAX) return NVFP4_ERR_UNSUPPORTED;
+    return NVFP4_OK;
+}
+
+// The new tokens of an append + attention call (nullptr: attention only).
+struct AppendArgs {
+    const void* x_k;
+    const void* x_v;
+    bool f32;
+    const int32_t* start_pos;
+    int32_t* new_lens;
+};
+
+nvfp4_status run_attention(const void* q, nvfp4_dtype q_dtype, int H_q, int B, int H_kv, int D,
+                           int S_max, const CacheView& c, const float* d_s_tensor_k,
+                           const float* d_s_tensor_v, const int32_t* d_seq_lens, float softmax_scale,
+                           float* out, void* workspace, size_t workspace_bytes, int32_t* d_status,
+                           nvfp4_stream_t stream, const AppendArgs* app = nullptr) {
+    const nvfp4_status pre = check_attention_args(q, q_dtype, H_q, B, H_kv, S_max, d_s_tensor_k,
+                                                  d_s_tensor_v, d_seq_lens, softmax_scale, out);
+    if (pre != NVFP4_OK || B == 0) return pre;
     const AttnWorkspace ws = attention_workspace(B, H_q, H_kv, D);
     if (workspace == nullptr || workspace_bytes < ws.total_bytes || !aligned16(workspace))
         return NVFP4_ERR_WORKSPACE;
@@ -116,6 +167,7 @@ nvfp4_status run_attention(const void* q, nvfp4_dtype q_dtype, int H_q, int B, i
     a.page_tokens = c.page_tokens;
     a.max_pages = c.max_pages;
     a.num_pages = c.num_pages;
+    a.wait_polls = g_wait_polls.load();
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     for (int b0 = 0; b0 < B; b0 += kMaxBatchPerLaunch) {
         const int nb = (B - b0) < kMaxBatchPerLaunch ? (B - b0) : kMaxBatchPerLaunch;
@@ -129,6 +181,14 @@ nvfp4_status run_attention(const void* q, nvfp4_dtype q_dtype, int H_q, int B, i
         a.seq_lens = d_seq_lens + b0;
         a.out = out + (size_t)b0 * H_q * D;
         a.counters = static_cast<int32_t*>(workspace) + (size_t)b0 * H_kv;
+        if (app != nullptr) {
+            const size_t xsz = app->f32 ? 4 : 2;
+            a.x_k_new = static_cast<const uint8_t*>(app->x_k) + (size_t)b0 * H_kv * D * xsz;
+            a.x_v_new = static_cast<const uint8_t*>(app->x_v) + (size_t)b0 * H_kv * D * xsz;
+            a.x_f32 = app->f32;
+            a.start_pos = app->start_pos + b0;
+            a.new_lens = app->new_lens != nullptr ? app->new_lens + b0 : nullptr;
+        }
         cudaError_t e = launch_decode_attention(a, s);
         if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     }
@@ -137,6 +197,21 @@ nvfp4_status run_attention(const void* q, nvfp4_dtype q_dtype, int H_q, int B, i
 
 
 }  // namespace
+
+namespace nvfp4kv {
+
+nvfp4_status attention_precheck(const void* q, nvfp4_dtype q_dtype, int H_q, const nvfp4_kv_plane* k,
+                                const nvfp4_kv_plane* v, const float* d_s_tensor_k,
+                                const float* d_s_tensor_v, const int32_t* d_seq_lens,
+                                float softmax_scale, const float* out) {
+    if (!plane_ok(k) || !plane_ok(v)) return NVFP4_ERR_INVALID_ARG;
+    if (k->B != v->B || k->H_kv != v->H_kv || k->S_max != v->S_max || k->D != v->D)
+        return NVFP4_ERR_INVALID_ARG;
+    return check_attention_args(q, q_dtype, H_q, k->B, k->H_kv, k->S_max, d_s_tensor_k, d_s_tensor_v,
+                                d_seq_lens, softmax_scale, out);
+}
+
+}  // namespace nvfp4kv
 
 extern "C" {
 
@@ -155,6 +230,11 @@ const char* nvfp4_status_string(int status) {
 }
 
 const char* nvfp4_version(void) { return "nvfp4kv 0.1.0 (sm_100a)"; }
+
+void nvfp4_set_wait_limit(int64_t polls) {
+    g_wait_polls.store(polls < 0 ? kDefaultWaitPolls
+                                 : (polls > (int64_t)UINT32_MAX ? UINT32_MAX : (uint32_t)polls));
+}
 
 size_t nvfp4_cache_bytes(int B, int H_kv, int S_max, int D) {
     if (B < 0 || H_kv <= 0 || S_max < 0 || D <= 0 || (D % 16) != 0) return 0;
@@ -273,6 +353,33 @@ nvfp4_status nvfp4_decode_attention(const void* q, nvfp4_dtype q_dtype, int H_q,
     c.seq_scale_bytes = plane_tok * (k->D / 16);
     return run_attention(q, q_dtype, H_q, k->B, k->H_kv, k->D, k->S_max, c, d_s_tensor_k, d_s_tensor_v,
                          d_seq_lens, softmax_scale, out, workspace, workspace_bytes, d_status, stream);
+}
+
+nvfp4_status nvfp4_decode_attention_append(const void* q, nvfp4_dtype q_dtype, int H_q,
+                                           const void* x_k_new, const void* x_v_new, nvfp4_dtype x_dtype,
+                                           const int32_t* d_start_pos, int32_t* d_new_lens,
+                                           const nvfp4_kv_plane* k, const nvfp4_kv_plane* v,
+                                           const float* d_s_tensor_k, const float* d_s_tensor_v,
+                                           float softmax_scale, float* out, void* workspace,
+                                           size_t workspace_bytes, int32_t* d_status,
+                                           nvfp4_stream_t stream) {
+    if (!plane_ok(k) || !plane_ok(v)) return NVFP4_ERR_INVALID_ARG;
+    if (k->B != v->B || k->H_kv != v->H_kv || k->S_max != v->S_max || k->D != v->D)
+        return NVFP4_ERR_INVALID_ARG;
+    if (x_dtype != NVFP4_IN_BF16 && x_dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
+    if (d_start_pos == nullptr || (d_new_lens != nullptr && d_new_lens == d_start_pos))
+        return NVFP4_ERR_INVALID_ARG;
+    if (k->B > 0 && (x_k_new == nullptr || x_v_new == nullptr || !aligned16(x_k_new) || !aligned16(x_v_new)))
+        return NVFP4_ERR_INVALID_ARG;
+    CacheView c{};
+    c.kc = k->codes; c.ks = k->scales; c.vc = v->codes; c.vs = v->scales;
+    const size_t plane_tok = (size_t)k->H_kv * k->S_max;
+    c.seq_code_bytes = plane_tok * (k->D / 2);
+    c.seq_scale_bytes = plane_tok * (k->D / 16);
+    AppendArgs app{x_k_new, x_v_new, x_dtype == NVFP4_IN_F32, d_start_pos, d_new_lens};
+    // the lengths come from d_start_pos (start + 1); it stands in for seq_lens in the checks
+    return run_attention(q, q_dtype, H_q, k->B, k->H_kv, k->D, k->S_max, c, d_s_tensor_k, d_s_tensor_v,
+                         d_start_pos, softmax_scale, out, workspace, workspace_bytes, d_status, stream, &app);
 }
 
 nvfp4_status nvfp4_decode_attention_paged(const void* q, nvfp4_dtype q_dtype, int H_q,

@@ -36,7 +36,31 @@ struct Params {
     // pool laid out [page][Hkv][page_tokens][...]; S_max = max_pages * page_tokens
     const int32_t* block_table;
     int page_tokens, max_pages, num_pages;
+    // sleeping polls (each up to 20 us) after which a pipeline wait of the
+    // tensor-core kernel gives up and reports NVFP4_ERR_TIMEOUT
+    uint32_t wait_polls;
+    // append + attention: with len_from_start the attention covers
+    // start_pos[b] + 1 tokens (seq_lens is not read); with x_k_new != nullptr
+    // as well (tensor-core kernel, contiguous planes) the kernel itself first
+    // quantizes one new token per sequence, x_k_new / x_v_new [B][1][Hkv][D]
+    // (bf16, or fp32 when x_f32), into slot start_pos[b] of the K and V planes
+    // (new_lens, if given, receives start_pos[b] + 1)
+    int len_from_start;
+    const void* x_k_new;
+    const void* x_v_new;
+    const int32_t* start_pos;
+    int32_t* new_lens;
+    int x_f32;
 };
+
+// Tokens to attend for sequence b: seq_lens[b], or start_pos[b] + 1 after an
+// append; clamped to [0, S_max] (the caller reports past-capacity).
+__device__ __forceinline__ int attended_len(const Params& p, int b, bool* out_of_range) {
+    const int L = p.len_from_start ? p.start_pos[b] + 1 : p.seq_lens[b];
+    const bool bad = L < 0 || L > p.S_max || (p.len_from_start && L < 1);
+    if (out_of_range) *out_of_range = bad;
+    return L < 0 ? 0 : (L > p.S_max ? p.S_max : L);
+}
 
 // Global tile index -> (sequence, head, first tile of the unit, length).
 struct Unit {
@@ -56,22 +80,40 @@ __host__ __device__ __forceinline__ Unit find_unit(const int32_t* prefix, const 
     u.b = lo;
     u.L = lens[lo];
     u.ntb = u.L > 0 ? (u.L + TILE - 1) / TILE : 1;
-    const int64_t r = gt - prefix[lo];
-    u.h = (int)(r / u.ntb);
+    // r < H_kv * ntb <= the launch's tile count < 2^31: a 32-bit division
+    // (a 64-bit one is a long software routine)
+    const uint32_t r = (uint32_t)(gt - prefix[lo]);
+    u.h = (int)(r / (uint32_t)u.ntb);
     u.U0 = prefix[lo] + (int64_t)u.h * u.ntb;
     u.U1 = u.U0 + u.ntb;
     (void)Hkv;
     return u;
 }
 
+// floor(a / n) for 0 <= a < 2^53 and 0 < n < 2^53.  The correctly rounded
+// double quotient is within one of the exact one (its error is below
+// a / n * 2^-53 < 1), and one integer step each way fixes it.  This replaces
+// the software routine of a 64-bit integer division, which costs a few
+// hundred cycles.
+__host__ __device__ __forceinline__ int64_t div_floor(int64_t a, int64_t n) {
+    int64_t q = (int64_t)((double)a / (double)n);
+    if (q * n > a) {
+        --q;
+    } else if ((q + 1) * n <= a) {
+        ++q;
+    }
+    return q;
+}
+
 // CTA c owns global tiles [range_start(c), range_start(c + 1)).
+// (c <= N < 2^16 and T < 2^31, so c * T < 2^47.)
 __host__ __device__ __forceinline__ int64_t range_start(int64_t c, int64_t T, int64_t N) {
-    return c * T / N;
+    return div_floor(c * T, N);
 }
 
 // CTA owning global tile t when T tiles are cut into N equal ranges.
 __host__ __device__ __forceinline__ int64_t cta_of(int64_t t, int64_t T, int64_t N) {
-    return ((t + 1) * N - 1) / T;
+    return div_floor((t + 1) * N - 1, T);
 }
 
 // Partial-result slot of CTA cc for a unit starting at global tile U0: a CTA

@@ -321,11 +321,9 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_attention_kern
             const int b = tid * per + i;
             int L = 0;
             if (b < B) {
-                L = p.seq_lens[b];
-                if (L < 0 || L > p.S_max) {
-                    if (blockIdx.x == 0) report(p.status, NVFP4_ERR_CAPACITY);
-                    L = L < 0 ? 0 : p.S_max;
-                }
+                bool bad;
+                L = attended_len(p, b, &bad);
+                if (bad && blockIdx.x == 0) report(p.status, NVFP4_ERR_CAPACITY);
                 sm.lens[b] = L;
             }
             tiles[i] = (b < B) ? p.Hkv * (L > 0 ? (L + kTile - 1) / kTile : 1) : 0;
@@ -687,14 +685,9 @@ template <int D, int NT, bool QF32>
 cudaError_t launch_instance(const Params& p, int grid, cudaStream_t stream) {
     auto kern = decode_attention_kernel<D, NT, QF32>;
     const int smem = (int)sizeof(Smem<D, NT>);
-    static int configured_device = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_device != dev) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        configured_device = dev;
-    }
+    static int configured[kMaxDevices] = {};
+    cudaError_t e0 = ensure_smem_attribute(reinterpret_cast<const void*>(kern), smem, configured);
+    if (e0 != cudaSuccess) return e0;
     kern<<<grid, kWarps * 32, smem, stream>>>(p);
     return cudaGetLastError();
 }
@@ -717,10 +710,30 @@ cudaError_t launch_decode_attention(const AttnLaunch& a, cudaStream_t stream) {
     p.page_tokens = a.page_tokens;
     p.max_pages = a.max_pages;
     p.num_pages = a.num_pages;
+    p.wait_polls = a.wait_polls;
+    p.len_from_start = a.start_pos != nullptr ? 1 : 0;
+    p.start_pos = a.start_pos;
+    p.new_lens = a.new_lens;
+    p.x_f32 = a.x_f32 ? 1 : 0;
+    p.x_k_new = nullptr;
+    p.x_v_new = nullptr;
     const bool two = p.g > 8;
     const int sms = device_sm_count();
-    if (a.D == 128 && !a.q_f32)   // fifth-generation tensor cores: the main path
+    if (a.D == 128 && !a.q_f32) {   // fifth-generation tensor cores: the main path
+        p.x_k_new = a.x_k_new;       // the kernel appends the new tokens itself
+        p.x_v_new = a.x_v_new;
         return launch_decode_attention_tc(p, sms, stream);
+    }
+    if (a.x_k_new != nullptr) {      // warp-MMA path: the append runs as its own launch first
+        nvfp4_kv_plane pk{}, pv{};
+        pk.codes = const_cast<uint8_t*>(a.kc); pk.scales = const_cast<uint8_t*>(a.ks);
+        pv.codes = const_cast<uint8_t*>(a.vc); pv.scales = const_cast<uint8_t*>(a.vs);
+        pk.B = pv.B = a.B; pk.H_kv = pv.H_kv = a.Hkv; pk.S_max = pv.S_max = a.S_max; pk.D = pv.D = a.D;
+        cudaError_t e = launch_quantize_append_kv(a.x_k_new, a.x_v_new, a.x_f32, 1, a.start_pos, a.new_lens,
+                                                  a.st_k, a.st_v, pk, pv, a.status, stream);
+        if (e != cudaSuccess) return e;
+        p.new_lens = nullptr;
+    }
     const int grid = kCtasPerSm * sms;   // warp-MMA kernel: fp32 queries or head_dim 64
     if (a.D == 128) {
         if (!two) return a.q_f32 ? launch_instance<128, 1, true>(p, grid, stream)

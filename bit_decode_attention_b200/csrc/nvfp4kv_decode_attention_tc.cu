@@ -8,25 +8,35 @@
 //     out[b][h] = softmax(q . K^T * scale) . V   over seq_lens[b] tokens.
 //
 // Work split: the (sequence, KV head, 128-token tile) list is cut into one
-// contiguous range per CTA, one CTA per SM (stream-K); a (sequence, head)
-// unit shared by several CTAs is merged by the last one to finish with it.
+// contiguous range per CTA, one CTA per SM (stream-K).  A (sequence, head)
+// unit that crosses a range boundary leaves one partial (O, m, l) per CTA in
+// the workspace; a second, small kernel (launched as a programmatic dependent
+// of this one, so it is resident before this grid ends) merges them.  The
+// attention kernel itself therefore has no atomics, counters or merge code.
 //
 // Inside a CTA every stage of a tile has its own warps, and the stages of
 // consecutive tiles overlap; they hand tiles to each other through
-// mbarriers (double-buffered operands), never through CTA-wide barriers:
+// mbarriers, never through CTA-wide barriers:
 //
 //   load warp   : bulk copies of K/V codes and scale bytes into a 4-stage ring
 //   dequant warps 0-3 and 8-11: thread t of group h = token t, head_dim half
 //                 h.  K codes -> signed FP8 K in tensor memory lane t (the A
 //                 operand of Q.K^T); V codes -> FP8 V^T in shared memory (the
-//                 MN-major A operand of P.V).  K and V^T have 5 buffers
-//   MMA warp    : S^T[t][n] = K . Q'^T,  O^T[d][n] += V^T . P^T
-//                 (a tcgen05 MMA costs about the same for any N up to 256:
-//                 the instruction count per tile, 4 + 4, sets the pace)
+//                 MN-major A operand of P.V)
+//   MMA thread  : a fixed schedule, one tile ahead on Q.K^T:
+//                   S^T(w+1) = K(w+1) . Q'^T,   then   O^T += V^T(w) . P^T(w)
+//                 four MMAs and one commit per product; every wait blocks on
+//                 one barrier (no polling of several)
 //   softmax 4-7 : thread t reads score row t, online softmax in base 2 with a
 //                 lazily raised running max, P as three E4M3 terms
 //                 p ~ t0 + t1/16 + t2/256 (MN-major B operand); at the end of
-//                 a unit thread d reads O^T row d and writes the output
+//                 a unit thread d reads O^T row d and writes the output row or
+//                 the split-K partial
+//
+// Four buffers of every kind: tile w uses K/S buffer w % 4 (tensor memory)
+// and V^T/P buffer w % 4 (shared memory).  One commit after Q.K^T(w) both
+// publishes S(w) and frees K(w); one after P.V(w) publishes O and frees V^T(w)
+// and P(w).
 //
 // The query operand Q' holds, per query row, an exact two-term E4M3 split of
 // the bf16 query scaled by a power of two: q * 2^e = hi + lo / 16, so the
@@ -48,31 +58,38 @@ constexpr int STAGE = TILE * (2 * kKB + 2 * kSB);     // 18432
 constexpr int OFF_VC = TILE * kKB;
 constexpr int OFF_KS = 2 * TILE * kKB;
 constexpr int OFF_VS = 2 * TILE * kKB + TILE * kSB;
-constexpr int kStages = 4;
-// operand buffers: K (tensor memory) and V^T (shared memory) let the dequant
-// warps run ahead of the softmax; S (tensor memory) lets Q.K^T run ahead
-constexpr int kKBuf = 5, kVBuf = 5, kSBuf = 3, kPBuf = 3;
+constexpr int kStages = 4;                            // bulk-copy ring
+constexpr int kBuf = 4;                               // K/S and V^T/P operand buffers
 constexpr int NTERM = 3;                              // E4M3 terms of P
 
-// warp roles
-constexpr int kSWarp0 = 4;                            // warps 4-7: softmax / output
-constexpr int kVWarp0 = 8;                            // warps 0-3 and 8-11: dequant
-constexpr int kLoadWarp = 12;
-constexpr int kMmaWarp = 13;
-constexpr int kThreads = 14 * 32;
-constexpr int kSoftmaxBar = 1;                        // named barrier of the softmax warps
+// warp roles, in warpgroups of four (warp w reaches tensor-memory lanes
+// 32 * (w % 4) .. +31, so every group covers the 128 token lanes):
+//   warps  0- 3  K dequant, head_dim  0-63      warps 16-19  V dequant, head_dim 64-127
+//   warps  4- 7  softmax group 0 (queries 0 .. NQ/2-1)
+//   warps  8-11  K dequant, head_dim 64-127     warps 20-23  softmax group 1 (NQ/2 .. NQ-1)
+//   warps 12-15  V dequant, head_dim  0-63      warp 24 loads, warp 25 MMAs (26-27 idle)
+constexpr int kS0Warp0 = 4;
+constexpr int kK1Warp0 = 8;
+constexpr int kV0Warp0 = 12;
+constexpr int kV1Warp0 = 16;
+constexpr int kS1Warp0 = 20;
+constexpr int kLoadWarp = 24;
+constexpr int kMmaWarp = 25;
+constexpr int kThreads = 28 * 32;
+// registers per thread after the prologue (setmaxnreg); the launch holds
+// kThreads x 72, and 128 x (2 x 112 + 4 x 56 + 56) = 64,512 of them
+constexpr uint32_t kRegsSoftmax = 112, kRegsDequant = 56, kRegsMisc = 56;
 
 constexpr uint32_t kWaitPolls = 1u << 16;             // sleeping polls (<= 20 us each) per wait
-constexpr uint32_t kMmaIdlePolls = 1u << 25;          // idle polls (~32 ns sleep each) of the MMA thread
 
 template <int NT>
 struct Cfg {
     static constexpr int NQ = 8 * NT;                 // query rows (padded GQA group)
     static constexpr int NS = 2 * NQ;                 // score columns: hi, lo
     static constexpr int NP = (NTERM * NQ + 15) / 16 * 16;   // P columns (MMA N), term-major
-    static constexpr uint32_t COL_K = 0;              // kKBuf buffers x 32 columns (4 FP8 each)
-    static constexpr uint32_t COL_S = 32 * kKBuf;     // kSBuf buffers x NS
-    static constexpr uint32_t COL_O = COL_S + kSBuf * NS;  // NP
+    static constexpr uint32_t COL_K = 0;              // kBuf buffers x 32 columns (4 FP8 each)
+    static constexpr uint32_t COL_S = 32 * kBuf;      // kBuf buffers x NS
+    static constexpr uint32_t COL_O = COL_S + kBuf * NS;   // NP
     static constexpr uint32_t kTmemCols = COL_O + NP <= 128 ? 128 : (COL_O + NP <= 256 ? 256 : 512);
     static_assert(COL_O + NP <= kTmemCols, "tensor memory columns");
 };
@@ -85,13 +102,13 @@ template <int NT>
 struct __align__(1024) Smem {
     using C = Cfg<NT>;
     uint8_t ring[kStages][STAGE];
-    uint8_t vt[kVBuf][128 * TILE];                        // V^T: (d/16)*2048 + (t/8)*128 + (t%8)*16 + d%16
-    uint8_t pb[kPBuf][C::NP * TILE];                      // P^T: (n/16)*2048 + (t/8)*128 + (t%8)*16 + n%16
+    uint8_t vt[kBuf][128 * TILE];                     // V^T: (d/16)*2048 + (t/8)*128 + (t%8)*16 + d%16
+    uint8_t pb[kBuf][C::NP * TILE];                   // P^T: (n/16)*2048 + (t/8)*128 + (t%8)*16 + n%16
     uint8_t qb[2][C::NS * 128];                       // Q':  (n/8)*1024 + (d/16)*128 + (n%8)*16 + d%16
     uint2 lut[2][128][kLutCopies];
     uint64_t full[kStages], empty[kStages];
-    uint64_t kfull[kKBuf], kempty[kKBuf], vfull[kVBuf], vtfree[kVBuf];
-    uint64_t sfull[kSBuf], sempty[kSBuf], pfull[kPBuf], pvdone[kPBuf];
+    uint64_t kfull[kBuf], qkdone[kBuf], sempty[kBuf];
+    uint64_t vfull[kBuf], pfull[kBuf], pvdone[kBuf];
     uint64_t qfull[2];
     uint64_t mma_done;
     int32_t lens[kMaxBatchPerLaunch];
@@ -99,12 +116,8 @@ struct __align__(1024) Smem {
     float cscale[2][C::NQ];
     float red[4][C::NQ];
     int32_t warp_tot[kThreads / 32];
-    CombineSmem comb;
+    int32_t warp_empty[kThreads / 32];
     uint32_t tmem_base;
-    int32_t n_sig;                                    // split units whose partial this CTA wrote
-    int32_t n_pend;                                   // units this CTA must merge at its end
-    int64_t sig_gt[2];
-    int64_t pend_gt[2];
     int32_t abort_flag;
 };
 
@@ -130,12 +143,12 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 }
 
 // Bounded wait of one thread: gives up when the CTA's abort flag is set or
-// after kWaitPolls sleeping polls (then sets the flag and reports a timeout).
+// after `polls` sleeping polls (then sets the flag and reports a timeout).
 // Inlined: a call would spill the live registers of the caller.
 __device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, int32_t* abort_flag,
-                                         int32_t* status) {
+                                         int32_t* status, uint32_t polls) {
     if (mbar_test_wait(bar, parity)) return true;
-    for (uint32_t i = 0; i < kWaitPolls; ++i) {
+    for (uint32_t i = 0; i < polls; ++i) {
         if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
         if (*reinterpret_cast<volatile int32_t*>(abort_flag)) return false;
     }
@@ -146,22 +159,23 @@ __device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, int32_t
 
 // The same for a whole warp; the result is warp-uniform.
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, int32_t* abort_flag,
-                                          int32_t* status) {
-    const bool ok = wait_one(bar, parity, abort_flag, status);
+                                          int32_t* status, uint32_t polls) {
+    const bool ok = wait_one(bar, parity, abort_flag, status, polls);
     return __all_sync(0xFFFFFFFFu, ok);
 }
 
 // the softmax warps' named barrier, plain and as an OR-reduction
-__device__ __forceinline__ void softmax_sync() {
-    asm volatile("bar.sync %0, 128;" ::"n"(kSoftmaxBar) : "memory");
+// (named barrier 1 + group, 128 threads each)
+__device__ __forceinline__ void softmax_sync(int bar_id) {
+    asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
 }
-__device__ __forceinline__ bool softmax_any(bool v) {
+__device__ __forceinline__ bool softmax_any(bool v, int bar_id) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
         "bar.red.or.pred po, %2, 128, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)v), "n"(kSoftmaxBar)
+        : "r"((uint32_t)v), "r"(bar_id)
         : "memory");
     return r != 0;
 }
@@ -178,7 +192,9 @@ __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t* r) {
 // N consecutive 32-bit columns of this thread's lane (N = 8, 16, 32)
 template <int N>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* r) {
-    if constexpr (N == 8) {
+    if constexpr (N == 4) {
+        tc::tmem_ld_x4(taddr, r);
+    } else if constexpr (N == 8) {
         tc::tmem_ld_x8(taddr, r);
     } else if constexpr (N == 16) {
         tc::tmem_ld_x16(taddr, r);
@@ -190,13 +206,35 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* r) {
 }
 template <int N>
 __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t* r) {
-    if constexpr (N == 8) {
+    if constexpr (N == 4) {
+        tc::tmem_st_x4(taddr, r);
+    } else if constexpr (N == 8) {
         tc::tmem_st_x8(taddr, r);
     } else {
         static_assert(N == 16, "columns");
         tc::tmem_st_x8(taddr, r);
         tc::tmem_st_x8(taddr + 8, r + 8);
     }
+}
+
+// Registers per thread of this warpgroup (all four warps execute it).
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Allow the dependent grid (the split-K merge) to be scheduled.
+__device__ __forceinline__ void launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the grids this one depends on have completed and their memory
+// operations are visible.
+__device__ __forceinline__ void wait_prerequisites() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // Three E4M3 terms of two non-negative weights (two bytes each, lo weight in
@@ -224,46 +262,49 @@ __device__ __forceinline__ void p_terms(float p0, float p1, uint32_t (&t)[NTERM]
 // ---------------------------------------------------------------------------
 template <int NT>
 struct QRaw {
-    static constexpr int PER = Cfg<NT>::NQ;           // bf16 elements per thread: 8 or 16
-    uint4 w[PER / 8];
+    static constexpr int PER = Cfg<NT>::NQ / 2;       // bf16 elements per thread: 4 or 8
+    uint32_t w[PER / 2];
 };
 
+// Query rows q0 .. q0 + NQ/2 - 1 of unit (b, h), by the 128 threads of one
+// softmax group: thread t holds row q0 + t / TPQ, head_dim d0 .. d0 + PER - 1.
 template <int NT>
-__device__ __forceinline__ void fetch_q(const Params& p, int b, int h, int t, QRaw<NT>& raw) {
+__device__ __forceinline__ void fetch_q(const Params& p, int b, int h, int q0, int t, QRaw<NT>& raw) {
     constexpr int PER = QRaw<NT>::PER;
     constexpr int TPQ = 128 / PER;                    // threads per query row
-    const int q = t / TPQ;
+    const int q = q0 + t / TPQ;
     const int d0 = (t % TPQ) * PER;
     const bool valid = q < p.g;
     const int64_t row = ((int64_t)b * p.Hq + (int64_t)h * p.g + (valid ? q : 0)) * 128 + d0;
-    const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.q) + row);
-#pragma unroll
-    for (int i = 0; i < PER / 8; ++i) raw.w[i] = valid ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+    const uint16_t* src = reinterpret_cast<const uint16_t*>(p.q) + row;
+    if constexpr (PER == 8) {
+        const uint4 v = valid ? __ldg(reinterpret_cast<const uint4*>(src)) : make_uint4(0, 0, 0, 0);
+        raw.w[0] = v.x; raw.w[1] = v.y; raw.w[2] = v.z; raw.w[3] = v.w;
+    } else {
+        const uint2 v = valid ? __ldg(reinterpret_cast<const uint2*>(src)) : make_uint2(0, 0);
+        raw.w[0] = v.x; raw.w[1] = v.y;
+    }
 }
 
 template <int NT>
 __device__ __forceinline__ void build_q(const Params& p, uint8_t* qb, float* cscale, const QRaw<NT>& raw,
-                                        int t) {
+                                        int q0, int t) {
     using C = Cfg<NT>;
     constexpr int PER = QRaw<NT>::PER;
     constexpr int TPQ = 128 / PER;
-    const int q = t / TPQ;
+    const int q = q0 + t / TPQ;
     const int d0 = (t % TPQ) * PER;
     float v[PER];
 #pragma unroll
-    for (int i = 0; i < PER / 8; ++i) {
-        const uint32_t w[4] = {raw.w[i].x, raw.w[i].y, raw.w[i].z, raw.w[i].w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            v[8 * i + 2 * k + 0] = __uint_as_float(w[k] << 16);
-            v[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-        }
+    for (int k = 0; k < PER / 2; ++k) {
+        v[2 * k + 0] = __uint_as_float(raw.w[k] << 16);
+        v[2 * k + 1] = __uint_as_float(raw.w[k] & 0xFFFF0000u);
     }
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < PER; ++i) amax = fmaxf(amax, fabsf(v[i]));
 #pragma unroll
-    for (int o = 1; o < TPQ; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    for (int o = 1; o < TPQ && o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
     int e = 0;
     if (amax > 0.0f && amax <= 3.4028234663852886e38f) {
         int ex;
@@ -287,15 +328,13 @@ __device__ __forceinline__ void build_q(const Params& p, uint8_t* qb, float* csc
         hw[i / 4] = h01 | (h23 << 16);
         lw[i / 4] = l01 | (l23 << 16);
     }
-    // K-major rows n = q (hi) and n = NQ + q (lo); d0 is a multiple of 8
+    // K-major rows n = q (hi) and n = NQ + q (lo); d0 is a multiple of 4
     const int nh = q, nl = C::NQ + q;
 #pragma unroll
-    for (int c = 0; c < PER / 8; ++c) {
-        const int d = d0 + 8 * c;
-        uint8_t* dh = qb + (nh / 8) * 1024 + (d / 16) * 128 + (nh % 8) * 16 + d % 16;
-        uint8_t* dl = qb + (nl / 8) * 1024 + (d / 16) * 128 + (nl % 8) * 16 + d % 16;
-        *reinterpret_cast<uint2*>(dh) = make_uint2(hw[2 * c], hw[2 * c + 1]);
-        *reinterpret_cast<uint2*>(dl) = make_uint2(lw[2 * c], lw[2 * c + 1]);
+    for (int c = 0; c < PER / 4; ++c) {
+        const int d = d0 + 4 * c;
+        *reinterpret_cast<uint32_t*>(qb + (nh / 8) * 1024 + (d / 16) * 128 + (nh % 8) * 16 + d % 16) = hw[c];
+        *reinterpret_cast<uint32_t*>(qb + (nl / 8) * 1024 + (d / 16) * 128 + (nl % 8) * 16 + d % 16) = lw[c];
     }
     if (t % TPQ == 0) cscale[q] = p.softmax_scale * kLog2e * __uint_as_float(pow2_bits(-e));
 }
@@ -311,7 +350,7 @@ __device__ __forceinline__ int tile_valid(const Unit& u, int64_t gt) {
 // Walk over the tiles with work (valid > 0) of a CTA range, in order.  The
 // segment ordinal counts every segment (unit) of the range, empty ones too.
 struct TileWalker {
-    int64_t seg_lo, seg_hi, gt, t_end;
+    int64_t seg_hi, gt, t_end;
     Unit u;
     int64_t last;                                     // the tile returned by next()
     int32_t j;                                        // its segment ordinal
@@ -319,7 +358,7 @@ struct TileWalker {
     bool fresh;
 
     __device__ __forceinline__ void start(int64_t t_begin, int64_t t_end_) {
-        seg_lo = seg_hi = gt = t_begin;
+        seg_hi = gt = t_begin;
         t_end = t_end_;
         j = -1;
         fresh = true;
@@ -338,7 +377,7 @@ struct TileWalker {
                 continue;
             }
             if (seg_hi >= t_end) return false;
-            seg_lo = seg_hi;
+            const int64_t seg_lo = seg_hi;
             u = find_unit<TILE>(prefix, lens, B, Hkv, seg_lo);
             seg_hi = u.U1 < t_end ? u.U1 : t_end;
             gt = seg_lo;
@@ -349,7 +388,55 @@ struct TileWalker {
 };
 
 // ---------------------------------------------------------------------------
-// the kernel
+// Fused append (a2-a4 for one token): every unit whose last tile lies in
+// [t_begin, t_end) gets its new token -- K and V, 8 blocks each, one lane per
+// block (lanes 0-7 K, 8-15 V) of warp (unit ordinal % warps) -- quantized with
+// the same block quantizer as nvfp4_kv_quantize_append and written at slot
+// start_pos[b].  A sequence whose slot is out of range is skipped (the
+// prologue reported it); a non-finite or non-positive tensor scale skips
+// everything with NVFP4_ERR_NONFINITE.  The writers then order their global
+// stores before the async proxy's bulk copies (the caller's CTA barrier
+// follows).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void append_new_tokens(const Params& p, const int32_t* prefix, const int32_t* lens,
+                                               int B, int64_t t_begin, int64_t t_end, float st_k,
+                                               float st_v, int warp, int lane) {
+    const bool ok_k = st_k > 0.0f && st_k <= 3.4028234663852886e38f;
+    const bool ok_v = st_v > 0.0f && st_v <= 3.4028234663852886e38f;
+    int ui = 0;
+    for (int64_t seg_lo = t_begin; seg_lo < t_end;) {
+        const Unit u = find_unit<TILE>(prefix, lens, B, p.Hkv, seg_lo);
+        if (u.U1 <= t_end) {
+            if (ui % (kThreads / 32) == warp && lane < 16) {
+                const int start = p.start_pos[u.b];
+                const bool is_v = lane >= 8;
+                const int blk = lane & 7;
+                const bool in_range = start >= 0 && start + 1 <= p.S_max;
+                if (in_range && (is_v ? ok_v : ok_k)) {
+                    float v[16];
+                    const int64_t elem = ((int64_t)u.b * p.Hkv + u.h) * 128 + 16 * blk;
+                    if (p.x_f32) load16<true>(is_v ? p.x_v_new : p.x_k_new, elem, v);
+                    else load16<false>(is_v ? p.x_v_new : p.x_k_new, elem, v);
+                    uint2 packed;
+                    const uint32_t sb = quantize_block(v, is_v ? st_v : st_k, packed);
+                    const int64_t slot = ((int64_t)u.b * p.Hkv + u.h) * p.S_max + start;
+                    uint8_t* codes = const_cast<uint8_t*>(is_v ? p.vc : p.kc);
+                    uint8_t* scales = const_cast<uint8_t*>(is_v ? p.vs : p.ks);
+                    *reinterpret_cast<uint2*>(codes + slot * 64 + 8 * blk) = packed;
+                    scales[slot * 8 + blk] = (uint8_t)sb;
+                    if (!is_v && blk == 0 && u.h == 0 && p.new_lens != nullptr) p.new_lens[u.b] = start + 1;
+                }
+                if (!(ok_k && ok_v) && lane == 0) report(p.status, NVFP4_ERR_NONFINITE);
+            }
+            ++ui;
+        }
+        seg_lo = u.U1 < t_end ? u.U1 : t_end;
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// the attention kernel
 // ---------------------------------------------------------------------------
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const Params p) {
@@ -364,6 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const int B = p.B;
+    const uint32_t polls = p.wait_polls;
     const float st_k = __ldg(p.st_k);                 // loads in flight during the prefix scan
     const float st_v = __ldg(p.st_v);
 
@@ -377,11 +465,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
             const int b = tid * per + i;
             int L = 0;
             if (b < B) {
-                L = p.seq_lens[b];
-                if (L < 0 || L > p.S_max) {
-                    if (blockIdx.x == 0) report(p.status, NVFP4_ERR_CAPACITY);
-                    L = L < 0 ? 0 : p.S_max;
-                }
+                bool bad;
+                L = attended_len(p, b, &bad);
+                if (bad && blockIdx.x == 0) report(p.status, NVFP4_ERR_CAPACITY);
                 sm.lens[b] = L;
             }
             tiles[i] = (b < B) ? p.Hkv * (L > 0 ? (L + TILE - 1) / TILE : 1) : 0;
@@ -413,6 +499,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
     const int64_t t_begin = range_start(c, T, N);
     const int64_t t_end = range_start(c + 1, T, N);
     if (t_begin >= t_end) return;
+    {
+        // every tile of a unit has work except the single tile of an empty
+        // sequence's unit: count those inside this CTA's range
+        constexpr int per = (kMaxBatchPerLaunch + kThreads - 1) / kThreads;
+        int empty = 0;
+#pragma unroll
+        for (int i = 0; i < per; ++i) {
+            const int b = tid * per + i;
+            if (b < B && sm.lens[b] == 0) {
+                const int64_t lo = sm.prefix[b] > t_begin ? sm.prefix[b] : t_begin;
+                const int64_t hi = (int64_t)sm.prefix[b] + p.Hkv < t_end ? (int64_t)sm.prefix[b] + p.Hkv : t_end;
+                empty += hi > lo ? (int)(hi - lo) : 0;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) empty += __shfl_xor_sync(0xFFFFFFFFu, empty, o);
+        if (lane == 0) sm.warp_empty[warp] = empty;
+    }
 
     // ---- tensor memory, barriers, lookup tables, zeroed P buffers ----
     if (warp == kMmaWarp) {
@@ -426,41 +530,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
     if (warp == kLoadWarp && lane == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.empty[s], 8);
+            mbar_init(&sm.empty[s], 16);
         }
-        for (int b = 0; b < kKBuf; ++b) {
+        for (int b = 0; b < kBuf; ++b) {
             mbar_init(&sm.kfull[b], 8);
-            mbar_init(&sm.kempty[b], 1);
-        }
-        for (int b = 0; b < kVBuf; ++b) {
+            mbar_init(&sm.qkdone[b], 1);
+            mbar_init(&sm.sempty[b], 8);
             mbar_init(&sm.vfull[b], 8);
-            mbar_init(&sm.vtfree[b], 1);
-        }
-        for (int b = 0; b < kSBuf; ++b) {
-            mbar_init(&sm.sfull[b], 1);
-            mbar_init(&sm.sempty[b], 4);
-        }
-        for (int b = 0; b < kPBuf; ++b) {
-            mbar_init(&sm.pfull[b], 4);
+            mbar_init(&sm.pfull[b], 8);
             mbar_init(&sm.pvdone[b], 1);
         }
-        mbar_init(&sm.qfull[0], 4);
-        mbar_init(&sm.qfull[1], 4);
+        mbar_init(&sm.qfull[0], 8);
+        mbar_init(&sm.qfull[1], 8);
         mbar_init(&sm.mma_done, 1);
         fence_mbar_init();
         sm.abort_flag = 0;
-        sm.n_sig = 0;
-        sm.n_pend = 0;
         // the first two tiles only: the CTA barrier below waits for this lane
-        while (load_w < 2u && load_walk.next(sm.prefix, sm.lens, B, p.Hkv)) {
+        // (in the fused append mode every copy waits for the new tokens)
+        while (p.x_k_new == nullptr && load_w < 2u && load_walk.next(sm.prefix, sm.lens, B, p.Hkv)) {
             issue_tile<128, TILE>(p, load_walk.u, load_walk.last, sm.ring[load_w], &sm.full[load_w]);
             ++load_w;
         }
     }
     QRaw<NT> q_first;                                 // query loads in flight during the table build
-    if (warp >= kSWarp0 && warp < kVWarp0) {
+    const int wg = warp >> 2;                          // warpgroup
+    const bool is_softmax = wg == kS0Warp0 / 4 || wg == kS1Warp0 / 4;
+    const int sgrp = wg == kS1Warp0 / 4 ? 1 : 0;       // softmax group
+    if (is_softmax) {
         const Unit u0 = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, t_begin);
-        fetch_q<NT>(p, u0.b, u0.h, tid - 32 * kSWarp0, q_first);
+        fetch_q<NT>(p, u0.b, u0.h, sgrp * (NQ / 2), 32 * (warp & 3) + lane, q_first);
     }
     if (tid < 256) {
         const int plane = tid >> 7;
@@ -481,16 +579,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
+    if (p.x_k_new != nullptr) {
+        // fused append: the CTA that owns a unit's last tile quantizes the
+        // unit's new token (slot L - 1) before any copy of that tile is issued
+        append_new_tokens(p, sm.prefix, sm.lens, B, t_begin, t_end, st_k, st_v, warp, lane);
+        __syncthreads();
+    }
     const uint32_t tbase = sm.tmem_base;
     int32_t* const abort_flag = &sm.abort_flag;
+    launch_dependents();                              // the merge grid may be scheduled now
+    int n_work = (int)(t_end - t_begin);              // tiles with work in this CTA's range
+#pragma unroll
+    for (int i = 0; i < kThreads / 32; ++i) n_work -= sm.warp_empty[i];
 
+    // each role sets its warpgroup's register count first (setmaxnreg); the
+    // loader's and the MMA warp's group also holds the two idle warps
+    if (wg == kLoadWarp / 4) {
+        regs_dec<kRegsMisc>();
+    }
     if (warp == kLoadWarp) {
         // ================= bulk copies into the ring =================
         if (lane == 0) {
             uint32_t w = load_w;                       // the first stages went out in the prologue
             while (load_walk.next(sm.prefix, sm.lens, B, p.Hkv)) {
                 const int s = (int)(w % kStages);
-                if (w >= (uint32_t)kStages && !wait_one(&sm.empty[s], ((w / kStages) - 1) & 1u, abort_flag, p.status))
+                if (w >= (uint32_t)kStages &&
+                    !wait_one(&sm.empty[s], ((w / kStages) - 1) & 1u, abort_flag, p.status, polls))
                     break;
                 issue_tile<128, TILE>(p, load_walk.u, load_walk.last, sm.ring[s], &sm.full[s]);
                 ++w;
@@ -505,170 +619,222 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
             }
         }
     } else if (warp == kMmaWarp) {
-        // ================= tensor-core MMAs (one thread) =================
-        // Q.K^T runs ahead of the softmax as far as the S buffers allow; P.V
-        // follows the softmax.  Both streams are polled, so neither waits
-        // behind the other.
-        if (lane == 0) {
-            const uint32_t idesc_qk = tc::idesc_e4m3(128, NS, false, false, false);
-            const uint32_t idesc_pv = tc::idesc_e4m3(128, C::NP, true, true, false);
-            TileWalker qk, pv;
-            qk.start(t_begin, t_end);
-            pv.start(t_begin, t_end);
-            bool qk_more = qk.next(sm.prefix, sm.lens, B, p.Hkv);
-            bool pv_more = pv.next(sm.prefix, sm.lens, B, p.Hkv);
-            uint32_t wq = 0, wp = 0;                   // work tiles issued per stream
-            int32_t q_seg = -1;                        // segment whose query operand is in place
-            uint32_t idle = 0;
-            bool ok = true;
-            while (ok && (qk_more || pv_more)) {
-                bool progress = false;
-                if (pv_more && wp < wq) {
-                    const int bv = (int)(wp % kVBuf), bp = (int)(wp % kPBuf);
-                    if (mbar_test_wait(&sm.vfull[bv], (wp / kVBuf) & 1u) &&
-                        mbar_test_wait(&sm.pfull[bp], (wp / kPBuf) & 1u)) {
-                        tc::fence_after_sync();
-                        const uint32_t va = tc::smem_addr(sm.vt[bv]);
-                        const uint32_t pa = tc::smem_addr(sm.pb[bp]);
-                        const bool first = pv.first;   // O restarts with each unit
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            tc::mma_e4m3_ss(tbase + C::COL_O, tc::smem_desc(va + ks * 512, 128, 2048),
-                                            tc::smem_desc(pa + ks * 512, 128, 2048), idesc_pv,
-                                            !first || ks > 0);
-                        tc::mma_commit(&sm.pvdone[bp]);
-                        tc::mma_commit(&sm.vtfree[bv]);
-                        ++wp;
-                        pv_more = pv.next(sm.prefix, sm.lens, B, p.Hkv);
-                        progress = true;
-                    }
-                }
-                if (qk_more) {
-                    const int bk = (int)(wq % kKBuf), bs = (int)(wq % kSBuf);
-                    const int32_t jq = qk.j;
-                    const bool q_ok = q_seg == jq || mbar_test_wait(&sm.qfull[jq & 1], (jq >> 1) & 1u);
-                    if (q_ok) q_seg = jq;
-                    if (q_ok && mbar_test_wait(&sm.kfull[bk], (wq / kKBuf) & 1u) &&
-                        (wq < (uint32_t)kSBuf || mbar_test_wait(&sm.sempty[bs], ((wq / kSBuf) - 1) & 1u))) {
-                        tc::fence_after_sync();
-                        const uint32_t qa = tc::smem_addr(sm.qb[jq & 1]);
-                        const uint32_t kcol = tbase + C::COL_K + 32 * bk;
-                        const uint32_t scol = tbase + C::COL_S + NS * bs;
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            tc::mma_e4m3_ts(scol, kcol + 8 * ks, tc::smem_desc(qa + ks * 256, 128, 1024),
-                                            idesc_qk, ks > 0);
-                        tc::mma_commit(&sm.sfull[bs]);
-                        tc::mma_commit(&sm.kempty[bk]);
-                        ++wq;
-                        qk_more = qk.next(sm.prefix, sm.lens, B, p.Hkv);
-                        progress = true;
-                    }
-                }
-                if (progress) {
-                    idle = 0;
-                } else {
-                    if (*reinterpret_cast<volatile int32_t*>(abort_flag)) break;
-                    if (++idle > kMmaIdlePolls) {
-                        atomicExch(abort_flag, 1);
-                        report(p.status, NVFP4_ERR_TIMEOUT);
-                        ok = false;
-                    }
-                    __nanosleep(32);
-                }
-            }
-            // every issued MMA must complete before tensor memory is released
-            tc::mma_commit(&sm.mma_done);
-            if (!mbar_wait_sleep(&sm.mma_done, 0, kWaitPolls)) report(p.status, NVFP4_ERR_TIMEOUT);
-        }
-        __syncwarp();
-    } else if (warp < kSWarp0 || warp >= kVWarp0) {
-        // ======== dequant: head_dim half h of the K and V rows of token t ========
-        const int h = warp >= kVWarp0 ? 1 : 0;            // head_dim [64h, 64h + 64)
-        const int t = tid - (h ? 32 * kVWarp0 : 0);        // token, tensor-memory lane
-        const uint32_t trow = tbase + ((uint32_t)(32 * (warp & 3)) << 16);
-        const int rot = (t >> 1) & 1;                      // V chunk order: fewer bank conflicts
-        const uint2* lut_k = &sm.lut[0][0][lane & (kLutCopies - 1)];
-        const uint2* lut_v = &sm.lut[1][0][lane & (kLutCopies - 1)];
-        uint32_t w = 0;
+        // ================= tensor-core MMAs =================
+        // The whole warp runs the schedule and its waits (every value stays
+        // warp-uniform); one elected lane issues each group of four MMAs
+        // together with its commit.
+        const uint32_t idesc_qk = tc::idesc_e4m3(128, NS, false, false, false);
+        const uint32_t idesc_pv = tc::idesc_e4m3(128, C::NP, true, true, false);
+        // descriptors of buffer 0; buffer b and k-step ks add to the
+        // start-address field (16-byte units, no carry out of its 14 bits)
+        const uint64_t qdesc0 = tc::smem_desc(tc::smem_addr(sm.qb[0]), 128, 1024);
+        const uint64_t vdesc0 = tc::smem_desc(tc::smem_addr(sm.vt[0]), 128, 2048);
+        const uint64_t pdesc0 = tc::smem_desc(tc::smem_addr(sm.pb[0]), 128, 2048);
+        constexpr uint64_t kQStep = (C::NS * 128) >> 4, kVStep = (128 * TILE) >> 4,
+                           kPStep = (C::NP * TILE) >> 4;
+        TileWalker walk;
+        walk.start(t_begin, t_end);
         bool ok = true;
-        for (int64_t seg_lo = t_begin; seg_lo < t_end && ok;) {
-            const Unit u = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, seg_lo);
-            const int64_t seg_hi = u.U1 < t_end ? u.U1 : t_end;
-            for (int64_t gt = seg_lo; gt < seg_hi && ok; ++gt) {
-                if (tile_valid(u, gt) <= 0) continue;
-                const int s = (int)(w % kStages);
-                const int bk = (int)(w % kKBuf), bv = (int)(w % kVBuf);
-                ok = wait_warp(&sm.full[s], (w / kStages) & 1u, abort_flag, p.status);
-                if (ok && w >= kKBuf)      // Q.K^T of tile w - kKBuf has read this K buffer
-                    ok = wait_warp(&sm.kempty[bk], ((w / kKBuf) - 1) & 1u, abort_flag, p.status);
-                if (!ok) break;
-                const uint8_t* st = sm.ring[s];
-                uint4 xk[2], xv[2];
+        int32_t q_seg = -1;                            // segment whose query operand is in place
+        // Q.K^T of tile wq: S(b) = K(b) . Q'^T, then commit to qkdone[b]
+        auto issue_qk = [&](uint32_t wq, int32_t jq) -> bool {
+            const int b = (int)(wq % kBuf);
+            const uint32_t ph = (wq / kBuf) & 1u;
+            if (q_seg != jq) {
+                if (!wait_warp(&sm.qfull[jq & 1], ((uint32_t)jq >> 1) & 1u, abort_flag, p.status, polls))
+                    return false;
+                q_seg = jq;
+            }
+            if (!wait_warp(&sm.kfull[b], ph, abort_flag, p.status, polls)) return false;
+            if (wq >= (uint32_t)kBuf && !wait_warp(&sm.sempty[b], ph ^ 1u, abort_flag, p.status, polls))
+                return false;
+            tc::fence_after_sync();
+            const uint64_t qd = qdesc0 + (uint64_t)(jq & 1) * kQStep;
+            const uint64_t bq[4] = {qd, qd + 16, qd + 32, qd + 48};
+            if (tc::elect_one())
+                tc::mma4_ts_commit(tbase + C::COL_S + NS * b, tbase + C::COL_K + 32 * b, bq, idesc_qk, 0u,
+                                   &sm.qkdone[b]);
+            __syncwarp();
+            return true;
+        };
+        // P.V of tile wp: O += V^T(b) . P^T(b), then commit to pvdone[b]; O
+        // restarts with the first tile of each unit
+        auto issue_pv = [&](uint32_t wp, bool first) -> bool {
+            const int b = (int)(wp % kBuf);
+            const uint32_t ph = (wp / kBuf) & 1u;
+            if (!wait_warp(&sm.vfull[b], ph, abort_flag, p.status, polls)) return false;
+            if (!wait_warp(&sm.pfull[b], ph, abort_flag, p.status, polls)) return false;
+            tc::fence_after_sync();
+            const uint64_t vd = vdesc0 + (uint64_t)b * kVStep;
+            const uint64_t pd = pdesc0 + (uint64_t)b * kPStep;
+            const uint64_t av[4] = {vd, vd + 32, vd + 64, vd + 96};
+            const uint64_t bp[4] = {pd, pd + 32, pd + 64, pd + 96};
+            if (tc::elect_one())
+                tc::mma4_ss_commit(tbase + C::COL_O, av, bp, idesc_pv, first ? 0u : 1u, &sm.pvdone[b]);
+            __syncwarp();
+            return true;
+        };
+        bool have = walk.next(sm.prefix, sm.lens, B, p.Hkv);
+        if (have) ok = issue_qk(0, walk.j);
+        uint32_t w = 0;
+        while (ok && have) {
+            const bool first = walk.first;             // of tile w
+            have = walk.next(sm.prefix, sm.lens, B, p.Hkv);
+            if (have) ok = issue_qk(w + 1, walk.j);
+            if (ok) ok = issue_pv(w, first);
+            ++w;
+        }
+        // every issued MMA must complete before tensor memory is released
+        if (tc::elect_one()) tc::mma_commit(&sm.mma_done);
+        __syncwarp();
+        if (!mbar_wait_sleep(&sm.mma_done, 0, kWaitPolls)) report(p.status, NVFP4_ERR_TIMEOUT);
+        __syncwarp();
+    } else if (wg == 0 || wg == kK1Warp0 / 4) {
+        // ======== K dequant: head_dim half h of token t's K row ========
+        // Software-pipelined: tile w's lookups, the publication of tile w - 1's
+        // tensor-memory stores, tile w + 1's raw data, then tile w's dequant
+        // and store -- each step's latency hides behind the next.
+        regs_dec<kRegsDequant>();
+        const int h = wg == 0 ? 0 : 1;                     // head_dim [64h, 64h + 64)
+        const int t = 32 * (warp & 3) + lane;              // token, tensor-memory lane
+        const uint32_t trow = tbase + ((uint32_t)(32 * (warp & 3)) << 16);
+        const uint2* lut_k = &sm.lut[0][0][lane & (kLutCopies - 1)];
+        uint4 xk[2];
+        uint32_t sk = 0;
+        // raw codes and scale bytes of tile w, then its ring stage is released
+        auto fetch = [&](int w) -> bool {
+            const int s = w % kStages;
+            if (!wait_warp(&sm.full[s], ((uint32_t)w / kStages) & 1u, abort_flag, p.status, polls)) return false;
+            const uint8_t* st = sm.ring[s];
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    xk[j] = *reinterpret_cast<const uint4*>(st + t * kKB + 32 * h + 16 * j);
-                    xv[j] = *reinterpret_cast<const uint4*>(st + OFF_VC + t * kKB + 32 * h + 16 * (j ^ rot));
-                }
-                const uint32_t sk = *reinterpret_cast<const uint32_t*>(st + OFF_KS + t * kSB + 4 * h);
-                const uint32_t sv = *reinterpret_cast<const uint32_t*>(st + OFF_VS + t * kSB + 4 * h);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.empty[s]);
-                // K: 64 codes -> 16 tensor-memory columns (4 FP8 each)
-                uint32_t kf[16];
+            for (int j = 0; j < 2; ++j) xk[j] = *reinterpret_cast<const uint4*>(st + t * kKB + 32 * h + 16 * j);
+            sk = *reinterpret_cast<const uint32_t*>(st + OFF_KS + t * kSB + 4 * h);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[s]);
+            return true;
+        };
+        bool ok = n_work > 0 && fetch(0);
+        int w = 0;
+        for (; ok && w < n_work; ++w) {
+            const int b = w % kBuf;
+            const uint32_t ph = ((uint32_t)w / kBuf) & 1u;
+            uint2 l[4];
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {              // 16 bytes = 32 codes = 2 blocks
-                    const uint2 l0 = lut_k[((sk >> (16 * j)) & 0x7F) * kLutCopies];
-                    const uint2 l1 = lut_k[((sk >> (16 * j + 8)) & 0x7F) * kLutCopies];
-                    dequant_word(xk[j].x, l0.x, l0.y, kf[8 * j + 0], kf[8 * j + 1]);
-                    dequant_word(xk[j].y, l0.x, l0.y, kf[8 * j + 2], kf[8 * j + 3]);
-                    dequant_word(xk[j].z, l1.x, l1.y, kf[8 * j + 4], kf[8 * j + 5]);
-                    dequant_word(xk[j].w, l1.x, l1.y, kf[8 * j + 6], kf[8 * j + 7]);
-                }
-                tmem_st_x16(trow + C::COL_K + 32 * bk + 16 * h, kf);
+            for (int i = 0; i < 4; ++i) l[i] = lut_k[((sk >> (8 * i)) & 0x7F) * kLutCopies];
+            const uint4 c0 = xk[0], c1 = xk[1];
+            if (w >= 1) {                                  // tile w - 1 is in tensor memory
                 tc::tmem_wait_st();
                 tc::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.kfull[bk]);  // Q.K^T may start before V is done
-                // P.V of tile w - kVBuf has read this V^T buffer
-                if (w >= kVBuf && !wait_warp(&sm.vtfree[bv], ((w / kVBuf) - 1) & 1u, abort_flag, p.status)) {
-                    ok = false;
-                    break;
-                }
-                // V: 64 codes -> 4 rows of 16 head_dim bytes of V^T
-                uint8_t* dst = sm.vt[bv] + (4 * h) * 2048 + (t / 8) * 128 + (t % 8) * 16;
+                if (lane == 0) mbar_arrive(&sm.kfull[(w - 1) % kBuf]);
+            }
+            if (w + 1 < n_work) ok = fetch(w + 1);
+            // Q.K^T of tile w - kBuf has read this K buffer
+            if (!ok || (w >= kBuf && !wait_warp(&sm.qkdone[b], ph ^ 1u, abort_flag, p.status, polls))) {
+                ok = false;
+                break;
+            }
+            // 64 codes -> 16 tensor-memory columns (4 FP8 each)
+            uint32_t kf[16];
+            dequant_word(c0.x, l[0].x, l[0].y, kf[0], kf[1]);
+            dequant_word(c0.y, l[0].x, l[0].y, kf[2], kf[3]);
+            dequant_word(c0.z, l[1].x, l[1].y, kf[4], kf[5]);
+            dequant_word(c0.w, l[1].x, l[1].y, kf[6], kf[7]);
+            dequant_word(c1.x, l[2].x, l[2].y, kf[8], kf[9]);
+            dequant_word(c1.y, l[2].x, l[2].y, kf[10], kf[11]);
+            dequant_word(c1.z, l[3].x, l[3].y, kf[12], kf[13]);
+            dequant_word(c1.w, l[3].x, l[3].y, kf[14], kf[15]);
+            tmem_st_x16(trow + C::COL_K + 32 * b + 16 * h, kf);
+        }
+        if (ok && n_work > 0) {
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.kfull[(n_work - 1) % kBuf]);
+        }
+    } else if (wg == kV0Warp0 / 4 || wg == kV1Warp0 / 4) {
+        // ======== V dequant: head_dim half h of token t's V row -> V^T ========
+        // Pipelined like the K warps: tile w - 1's V^T stores are published
+        // (proxy fence, arrive) one step later, while tile w's lookups fly.
+        regs_dec<kRegsDequant>();
+        const int h = wg == kV0Warp0 / 4 ? 0 : 1;
+        const int t = 32 * (warp & 3) + lane;              // token
+        const int rot = (t >> 1) & 1;                      // chunk order: fewer bank conflicts
+        const uint2* lut_v = &sm.lut[1][0][lane & (kLutCopies - 1)];
+        uint4 xv[2];
+        uint32_t sv = 0;
+        auto fetch = [&](int w) -> bool {
+            const int s = w % kStages;
+            if (!wait_warp(&sm.full[s], ((uint32_t)w / kStages) & 1u, abort_flag, p.status, polls)) return false;
+            const uint8_t* st = sm.ring[s];
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int cc = j ^ rot;                // head_dim 64h + 32cc .. +31
-                    const uint2 l0 = lut_v[((sv >> (16 * cc)) & 0x7F) * kLutCopies];
-                    const uint2 l1 = lut_v[((sv >> (16 * cc + 8)) & 0x7F) * kLutCopies];
-                    uint4 o0, o1;
-                    dequant_word(xv[j].x, l0.x, l0.y, o0.x, o0.y);
-                    dequant_word(xv[j].y, l0.x, l0.y, o0.z, o0.w);
-                    dequant_word(xv[j].z, l1.x, l1.y, o1.x, o1.y);
-                    dequant_word(xv[j].w, l1.x, l1.y, o1.z, o1.w);
-                    *reinterpret_cast<uint4*>(dst + (2 * cc) * 2048) = o0;
-                    *reinterpret_cast<uint4*>(dst + (2 * cc + 1) * 2048) = o1;
-                }
+            for (int j = 0; j < 2; ++j)
+                xv[j] = *reinterpret_cast<const uint4*>(st + OFF_VC + t * kKB + 32 * h + 16 * (j ^ rot));
+            sv = *reinterpret_cast<const uint32_t*>(st + OFF_VS + t * kSB + 4 * h);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[s]);
+            return true;
+        };
+        bool ok = n_work > 0 && fetch(0);
+        int w = 0;
+        for (; ok && w < n_work; ++w) {
+            const int b = w % kBuf;
+            const uint32_t ph = ((uint32_t)w / kBuf) & 1u;
+            // lookup words of chunk j (head_dim 64h + 32(j ^ rot) ..): its two blocks
+            uint2 l[4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int cc = j ^ rot;
+                l[2 * j] = lut_v[((sv >> (16 * cc)) & 0x7F) * kLutCopies];
+                l[2 * j + 1] = lut_v[((sv >> (16 * cc + 8)) & 0x7F) * kLutCopies];
+            }
+            const uint4 c[2] = {xv[0], xv[1]};
+            if (w >= 1) {                                  // tile w - 1's V^T is in shared memory
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.vfull[bv]);
-                ++w;
+                if (lane == 0) mbar_arrive(&sm.vfull[(w - 1) % kBuf]);
             }
-            seg_lo = seg_hi;
+            if (w + 1 < n_work) ok = fetch(w + 1);
+            // P.V of tile w - kBuf has read this V^T buffer
+            if (!ok || (w >= kBuf && !wait_warp(&sm.pvdone[b], ph ^ 1u, abort_flag, p.status, polls))) {
+                ok = false;
+                break;
+            }
+            // 64 codes -> 4 rows of 16 head_dim bytes of V^T
+            uint8_t* dst = sm.vt[b] + (4 * h) * 2048 + (t / 8) * 128 + (t % 8) * 16;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int cc = j ^ rot;
+                uint4 o0, o1;
+                dequant_word(c[j].x, l[2 * j].x, l[2 * j].y, o0.x, o0.y);
+                dequant_word(c[j].y, l[2 * j].x, l[2 * j].y, o0.z, o0.w);
+                dequant_word(c[j].z, l[2 * j + 1].x, l[2 * j + 1].y, o1.x, o1.y);
+                dequant_word(c[j].w, l[2 * j + 1].x, l[2 * j + 1].y, o1.z, o1.w);
+                *reinterpret_cast<uint4*>(dst + (2 * cc) * 2048) = o0;
+                *reinterpret_cast<uint4*>(dst + (2 * cc + 1) * 2048) = o1;
+            }
         }
-    } else {
-        // ================= softmax, P, output (warps 4-7) =================
-        const int t = tid - 32 * kSWarp0;                  // token of the score row; head_dim of O
-        const int sw = warp - kSWarp0;
+        if (ok && n_work > 0) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.vfull[(n_work - 1) % kBuf]);
+        }
+    } else if (is_softmax) {
+        // ============ softmax, P, output: group sgrp owns queries q0 .. q0 + NH - 1 ============
+        regs_inc<kRegsSoftmax>();
+        constexpr int NH = NQ / 2;
+        const int q0 = sgrp * NH;
+        const int bar_id = 1 + sgrp;
+        const int sw = warp & 3;                           // lane quadrant
+        const int t = 32 * sw + lane;                      // token of the score row; head_dim of O
         const uint32_t trow = tbase + ((uint32_t)(32 * sw) << 16);
         bool aborted = false;
         uint32_t w = 0;
         uint32_t j = 0;
         {   // query operand of the first unit (loads issued in the prologue)
-            build_q<NT>(p, sm.qb[0], sm.cscale[0], q_first, t);
+            build_q<NT>(p, sm.qb[0], sm.cscale[0], q_first, q0, t);
             fence_proxy_async_smem();
-            softmax_sync();
+            softmax_sync(bar_id);
             if (lane == 0) mbar_arrive(&sm.qfull[0]);
         }
         for (int64_t seg_lo = t_begin; seg_lo < t_end; ++j) {
@@ -678,12 +844,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
             QRaw<NT> qnext;
             if (has_next) {                                // loads in flight during this segment
                 const Unit un = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, seg_hi);
-                fetch_q<NT>(p, un.b, un.h, t, qnext);
+                fetch_q<NT>(p, un.b, un.h, q0, t, qnext);
             }
-            float cs[NQ], m_run[NQ], l_run[NQ];
+            float cs[NH], m_run[NH], l_run[NH];
 #pragma unroll
-            for (int q = 0; q < NQ; ++q) {
-                cs[q] = sm.cscale[j & 1u][q];
+            for (int q = 0; q < NH; ++q) {
+                cs[q] = sm.cscale[j & 1u][q0 + q];
                 m_run[q] = -INFINITY;
                 l_run[q] = 0.0f;
             }
@@ -691,73 +857,77 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
             for (int64_t gt = seg_lo; gt < seg_hi; ++gt) {
                 const int valid = tile_valid(u, gt);
                 if (valid <= 0) continue;
-                const int bs = (int)(w % kSBuf), bp = (int)(w % kPBuf);
-                float s[NQ];
-                if (!aborted && !wait_warp(&sm.sfull[bs], (w / kSBuf) & 1u, abort_flag, p.status)) aborted = true;
+                const int b = (int)(w % kBuf);
+                const uint32_t ph = (w / kBuf) & 1u;
+                float s[NH];
+                if (!aborted && !wait_warp(&sm.qkdone[b], ph, abort_flag, p.status, polls)) aborted = true;
                 if (!aborted) {
                     tc::fence_after_sync();
-                    uint32_t r[NS];
-                    tmem_ld_cols<NS>(trow + C::COL_S + NS * bs, r);
+                    uint32_t rh[NH], rl[NH];
+                    tmem_ld_cols<NH>(trow + C::COL_S + NS * b + q0, rh);
+                    tmem_ld_cols<NH>(trow + C::COL_S + NS * b + NQ + q0, rl);
                     tc::tmem_wait_ld();
                     tc::fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.sempty[bs]);
+                    if (lane == 0) mbar_arrive(&sm.sempty[b]);
                     const bool live = t < valid;
 #pragma unroll
-                    for (int q = 0; q < NQ; ++q)
-                        s[q] = live ? fmaf(__uint_as_float(r[NQ + q]), 0.0625f, __uint_as_float(r[q])) * cs[q]
+                    for (int q = 0; q < NH; ++q)
+                        s[q] = live ? fmaf(__uint_as_float(rl[q]), 0.0625f, __uint_as_float(rh[q])) * cs[q]
                                     : -INFINITY;
                 } else {
 #pragma unroll
-                    for (int q = 0; q < NQ; ++q) s[q] = -INFINITY;
+                    for (int q = 0; q < NH; ++q) s[q] = -INFINITY;
                 }
                 bool need = false;
 #pragma unroll
-                for (int q = 0; q < NQ; ++q) need |= s[q] > m_run[q] + kRescaleSlack;
-                if (softmax_any(need)) {
+                for (int q = 0; q < NH; ++q) need |= s[q] > m_run[q] + kRescaleSlack;
+                if (softmax_any(need, bar_id)) {
                     // raise the running max to the tile max (per query over the 128
-                    // tokens), rescale l and O
+                    // tokens), rescale l and this group's O columns
 #pragma unroll
-                    for (int q = 0; q < NQ; ++q) {
+                    for (int q = 0; q < NH; ++q) {
                         float mx = s[q];
 #pragma unroll
                         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-                        if (lane == 0) sm.red[sw][q] = mx;
+                        if (lane == 0) sm.red[sw][q0 + q] = mx;
                     }
-                    softmax_sync();
-                    float f[NQ];
+                    softmax_sync(bar_id);
+                    float f[NH];
 #pragma unroll
-                    for (int q = 0; q < NQ; ++q) {
-                        const float mt = fmaxf(fmaxf(sm.red[0][q], sm.red[1][q]), fmaxf(sm.red[2][q], sm.red[3][q]));
+                    for (int q = 0; q < NH; ++q) {
+                        const float mt = fmaxf(fmaxf(sm.red[0][q0 + q], sm.red[1][q0 + q]),
+                                               fmaxf(sm.red[2][q0 + q], sm.red[3][q0 + q]));
                         const float mn = fmaxf(m_run[q], mt);
                         f[q] = (m_run[q] == -INFINITY) ? 0.0f : fast_exp2(m_run[q] - mn);
                         m_run[q] = mn;
                         l_run[q] *= f[q];
                     }
-                    softmax_sync();                        // red is reused
+                    softmax_sync(bar_id);                  // red is reused
                     if (any_pv && !aborted) {
                         // the previous P.V must have landed in O before it is rescaled
                         const uint32_t v = w - 1;
-                        if (!wait_warp(&sm.pvdone[v % kPBuf], (v / kPBuf) & 1u, abort_flag, p.status)) aborted = true;
+                        if (!wait_warp(&sm.pvdone[v % kBuf], (v / kBuf) & 1u, abort_flag, p.status, polls))
+                            aborted = true;
                         if (!aborted) {
                             tc::fence_after_sync();
 #pragma unroll
                             for (int k = 0; k < NTERM; ++k) {
-                                uint32_t r[NQ];
-                                tmem_ld_cols<NQ>(trow + C::COL_O + k * NQ, r);
+                                uint32_t r[NH];
+                                tmem_ld_cols<NH>(trow + C::COL_O + k * NQ + q0, r);
                                 tc::tmem_wait_ld();
 #pragma unroll
-                                for (int q = 0; q < NQ; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * f[q]);
-                                tmem_st_cols<NQ>(trow + C::COL_O + k * NQ, r);
+                                for (int q = 0; q < NH; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * f[q]);
+                                tmem_st_cols<NH>(trow + C::COL_O + k * NQ + q0, r);
                             }
                             tc::tmem_wait_st();
                         }
                     }
                 }
-                // P terms of this token for every query: column n = k * NQ + q
-                uint32_t tw[NTERM][NQ / 4];
+                // P terms of this token for this group's queries: column n = k * NQ + q0 + q
+                uint32_t tw[NTERM][NH / 4];
 #pragma unroll
-                for (int q = 0; q < NQ; q += 4) {
+                for (int q = 0; q < NH; q += 4) {
                     uint32_t ta[NTERM], tb[NTERM];
                     float pq[4];
 #pragma unroll
@@ -770,26 +940,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
 #pragma unroll
                     for (int k = 0; k < NTERM; ++k) tw[k][q / 4] = ta[k] | (tb[k] << 16);
                 }
-                if (!aborted && w >= kPBuf &&
-                    !wait_warp(&sm.pvdone[bp], ((w / kPBuf) - 1) & 1u, abort_flag, p.status))
+                // P.V of tile w - kBuf has read this P buffer
+                if (!aborted && w >= (uint32_t)kBuf &&
+                    !wait_warp(&sm.pvdone[b], ph ^ 1u, abort_flag, p.status, polls))
                     aborted = true;
                 if (!aborted) {
-                    uint8_t* dst = sm.pb[bp] + (t / 8) * 128 + (t % 8) * 16;
+                    uint8_t* dst = sm.pb[b] + (t / 8) * 128 + (t % 8) * 16;
 #pragma unroll
                     for (int k = 0; k < NTERM; ++k) {
-                        const int n = k * NQ;
-                        if constexpr (NQ == 8) {
+                        const int n = k * NQ + q0;
+                        if constexpr (NH == 4) {
+                            *reinterpret_cast<uint32_t*>(dst + (n / 16) * 2048 + (n % 16)) = tw[k][0];
+                        } else {
                             *reinterpret_cast<uint2*>(dst + (n / 16) * 2048 + (n % 16)) =
                                 make_uint2(tw[k][0], tw[k][1]);
-                        } else {
-                            *reinterpret_cast<uint4*>(dst + (n / 16) * 2048) =
-                                make_uint4(tw[k][0], tw[k][1], tw[k][2], tw[k][3]);
                         }
                     }
                     fence_proxy_async_smem();
                     tc::fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.pfull[bp]);
+                    if (lane == 0) mbar_arrive(&sm.pfull[b]);
                 }
                 any_pv = true;
                 ++w;
@@ -797,29 +967,30 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
 
             // ---- segment end ----
             if (has_next) {
-                // query operand of the next unit; its buffer was last read by the
+                // query rows of the next unit; their buffer was last read by the
                 // Q.K^T MMAs of the unit before this one, all complete by now
-                build_q<NT>(p, sm.qb[(j + 1) & 1u], sm.cscale[(j + 1) & 1u], qnext, t);
+                build_q<NT>(p, sm.qb[(j + 1) & 1u], sm.cscale[(j + 1) & 1u], qnext, q0, t);
                 fence_proxy_async_smem();
-                softmax_sync();
+                softmax_sync(bar_id);
                 if (lane == 0) mbar_arrive(&sm.qfull[(j + 1) & 1u]);
             }
-            float o[NQ];
+            float o[NH];
 #pragma unroll
-            for (int q = 0; q < NQ; ++q) o[q] = 0.0f;
+            for (int q = 0; q < NH; ++q) o[q] = 0.0f;
             if (any_pv && !aborted) {
                 const uint32_t v = w - 1;
-                if (!wait_warp(&sm.pvdone[v % kPBuf], (v / kPBuf) & 1u, abort_flag, p.status)) aborted = true;
+                if (!wait_warp(&sm.pvdone[v % kBuf], (v / kBuf) & 1u, abort_flag, p.status, polls))
+                    aborted = true;
                 if (!aborted) {
                     tc::fence_after_sync();
                     float scale = 1.0f;
 #pragma unroll
                     for (int k = 0; k < NTERM; ++k) {
-                        uint32_t r[NQ];
-                        tmem_ld_cols<NQ>(trow + C::COL_O + k * NQ, r);
+                        uint32_t r[NH];
+                        tmem_ld_cols<NH>(trow + C::COL_O + k * NQ + q0, r);
                         tc::tmem_wait_ld();
 #pragma unroll
-                        for (int q = 0; q < NQ; ++q) o[q] = fmaf(__uint_as_float(r[q]), scale, o[q]);
+                        for (int q = 0; q < NH; ++q) o[q] = fmaf(__uint_as_float(r[q]), scale, o[q]);
                         scale *= 0.0625f;
                     }
                     tc::fence_before_sync();
@@ -827,45 +998,42 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
             }
             // l over the 128 tokens (per-thread partials; the running max is shared)
 #pragma unroll
-            for (int q = 0; q < NQ; ++q) {
+            for (int q = 0; q < NH; ++q) {
                 float l = l_run[q];
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, off);
-                if (lane == 0) sm.red[sw][q] = l;
+                if (lane == 0) sm.red[sw][q0 + q] = l;
             }
-            softmax_sync();
-            float lt[NQ];
+            softmax_sync(bar_id);
+            float lt[NH];
 #pragma unroll
-            for (int q = 0; q < NQ; ++q) lt[q] = (sm.red[0][q] + sm.red[1][q]) + (sm.red[2][q] + sm.red[3][q]);
+            for (int q = 0; q < NH; ++q)
+                lt[q] = (sm.red[0][q0 + q] + sm.red[1][q0 + q]) + (sm.red[2][q0 + q] + sm.red[3][q0 + q]);
 
             const bool whole = (u.U0 >= t_begin) && (u.U1 <= t_end);
             const int g = p.g;
-            const int64_t slot_floats = partial_slot_floats(g, 128);
             if (whole) {
 #pragma unroll
-                for (int q = 0; q < NQ; ++q)
-                    if (q < g)
-                        p.out[((int64_t)u.b * p.Hq + (int64_t)u.h * g + q) * 128 + t] =
+                for (int q = 0; q < NH; ++q)
+                    if (q0 + q < g)
+                        p.out[((int64_t)u.b * p.Hq + (int64_t)u.h * g + q0 + q) * 128 + t] =
                             (lt[q] > 0.0f) ? o[q] / lt[q] : 0.0f;
             } else {
-                float* part = p.partials + partial_slot(c, u.U0, T, N) * slot_floats;
+                // split unit: this CTA's partial; the merge kernel combines them
+                float* part = p.partials + partial_slot(c, u.U0, T, N) * partial_slot_floats(g, 128);
 #pragma unroll
-                for (int q = 0; q < NQ; ++q)
-                    if (q < g) part[q * 128 + t] = o[q];
+                for (int q = 0; q < NH; ++q)
+                    if (q0 + q < g) part[(q0 + q) * 128 + t] = o[q];
                 if (t == 0) {
 #pragma unroll
-                    for (int q = 0; q < NQ; ++q)
-                        if (q < g) {
-                            part[g * 128 + q] = m_run[q];
-                            part[g * 128 + g + q] = lt[q];
+                    for (int q = 0; q < NH; ++q)
+                        if (q0 + q < g) {
+                            part[g * 128 + q0 + q] = m_run[q];
+                            part[g * 128 + g + q0 + q] = lt[q];
                         }
                 }
-                // arrival is counted after the roles finish, so that the
-                // atomic (and the wait for its release) stays off this CTA's
-                // tile pipeline; a CTA splits at most its first and last unit
-                if (t == 0) sm.sig_gt[sm.n_sig++] = u.U0;
             }
-            softmax_sync();
+            softmax_sync(bar_id);
             seg_lo = seg_hi;
         }
     }
@@ -875,31 +1043,147 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
     __syncthreads();
     tc::fence_after_sync();
     if (warp == kMmaWarp) tc::tmem_dealloc(tbase, C::kTmemCols);
+}
 
-    // ---- split-K: count this CTA's arrival at each split unit (one lane per
-    // unit, atomics in flight together); the last to arrive merges the unit
-    // on every thread ----
-    if (warp == 0) {
-        const int n_sig = sm.n_sig;
-        bool last = false;
-        int64_t gt = 0;
-        if (lane < n_sig) {
-            gt = sm.sig_gt[lane];
-            const Unit u = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, gt);
-            const int prev = arrive_split_unit(&p.counters[(int64_t)u.b * p.Hkv + u.h]);
-            last = prev == unit_contributors(u.U0, u.U1, T, N) - 1;
+// ---------------------------------------------------------------------------
+// Split-K merge of the units the attention grid left in partials:
+//     out = sum_j w_j O_j / sum_j w_j l_j,   w_j = 2^(m_j - M),  M = max_j m_j
+// over the contributors j of a unit (m in base-2 score units).  One work item
+// is (unit b * H_kv + h, query q of the group), items spread round-robin over
+// the CTAs; an item whose unit lies inside one attention CTA's range is
+// skipped (that CTA wrote the output itself); otherwise thread d merges
+// head_dim element d.  The grid is a programmatic dependent of the attention
+// grid: it may become resident early, and griddepcontrol.wait holds it until
+// every attention CTA has finished and its partial stores are visible.
+// ---------------------------------------------------------------------------
+constexpr int kMergeThreads = 128;
+constexpr int kMergeBatch = 8;                        // O loads in flight per thread
+
+__device__ __forceinline__ float merge_block_max(float v, float* red, int warp, int lane) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    const float r = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    __syncthreads();
+    return r;
+}
+__device__ __forceinline__ float merge_block_sum(float v, float* red, int warp, int lane) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    const float r = (red[0] + red[1]) + (red[2] + red[3]);
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(kMergeThreads, 8) merge_split_units_kernel(const Params p, int n_attn) {
+    __shared__ int32_t s_lens[kMaxBatchPerLaunch];
+    __shared__ int32_t s_prefix[kMaxBatchPerLaunch + 1];
+    __shared__ int32_t s_warp_tot[kMergeThreads / 32];
+    __shared__ float s_w[kMergeThreads];
+    __shared__ float s_red[kMergeThreads / 32];
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int B = p.B;
+    // the lengths are final before the attention grid starts (stream order),
+    // so the split is recomputed while that grid still runs
+    {
+        constexpr int per = (kMaxBatchPerLaunch + kMergeThreads - 1) / kMergeThreads;
+        int tiles[per];
+        int run = 0;
+#pragma unroll
+        for (int i = 0; i < per; ++i) {
+            const int b = tid * per + i;
+            int L = 0;
+            if (b < B) {
+                L = attended_len(p, b, nullptr);
+                s_lens[b] = L;
+            }
+            tiles[i] = (b < B) ? p.Hkv * (L > 0 ? (L + TILE - 1) / TILE : 1) : 0;
+            run += tiles[i];
         }
-        const uint32_t lm = __ballot_sync(0xFFFFFFFFu, last);
-        if (last) sm.pend_gt[__popc(lm & ((1u << lane) - 1u))] = gt;
-        if (lane == 0) sm.n_pend = __popc(lm);
+        int incl = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) s_warp_tot[warp] = incl;
+        __syncthreads();
+        int before = 0;
+        for (int w = 0; w < warp; ++w) before += s_warp_tot[w];
+        int acc = before + incl - run;
+#pragma unroll
+        for (int i = 0; i < per; ++i) {
+            const int b = tid * per + i;
+            if (b < B) s_prefix[b] = acc;
+            acc += tiles[i];
+        }
+        if (tid == kMergeThreads - 1) s_prefix[B] = acc;
     }
     __syncthreads();
-    const int n_pend = sm.n_pend;
-    for (int i = 0; i < n_pend; ++i) {
-        const Unit u = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, sm.pend_gt[i]);
-        combine_partials<128, NT, kThreads, 0>(p, sm.comb, u, T, N, partial_slot_floats(p.g, 128), tid,
-                                               warp, lane);
-        if (tid == 0) atomicExch(&p.counters[(int64_t)u.b * p.Hkv + u.h], 0);
+    wait_prerequisites();                             // partials are complete and visible from here
+    const int64_t T = s_prefix[B];
+    const int64_t N = n_attn;
+    const int g = p.g;
+    const int64_t slot_floats = partial_slot_floats(g, 128);
+    const bool dense = T >= N;                        // every CTA range non-empty
+    const int n_items = B * p.Hkv * g;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int ui = item / g;                           // unit b * H_kv + h
+        const int q = item - ui * g;
+        const int b = ui / p.Hkv;
+        Unit u;
+        u.b = b;
+        u.h = ui - b * p.Hkv;
+        u.L = s_lens[b];
+        u.ntb = u.L > 0 ? (u.L + TILE - 1) / TILE : 1;
+        u.U0 = s_prefix[b] + (int64_t)u.h * u.ntb;
+        u.U1 = u.U0 + u.ntb;
+        const int64_t c = cta_of(u.U0, T, N);              // first contributor
+        if (cta_of(u.U1 - 1, T, N) == c) continue;         // inside one CTA's range: not split
+        const int ncc = unit_contributors(u.U0, u.U1, T, N);
+        const bool first_odd = range_start(c, T, N) < u.U0;   // the unit is c's second unit
+        // dense ranges: contributor j is CTA c + j (slot 2(c + j), or 2c + 1 for
+        // j = 0 when the unit is c's second unit); otherwise the closed form
+        const float* base = p.partials + 2 * c * slot_floats;
+        auto part_of = [&](int j) -> const float* {
+            if (dense) return base + (2 * (int64_t)j + ((j == 0 && first_odd) ? 1 : 0)) * slot_floats;
+            return p.partials + contributor_slot(j, u.U0, c, first_odd, dense, T, N) * slot_floats;
+        };
+        float mx = -INFINITY;
+        for (int j = tid; j < ncc; j += kMergeThreads) mx = fmaxf(mx, __ldcg(part_of(j) + g * 128 + q));
+        const float M = merge_block_max(mx, s_red, warp, lane);
+        float acc = 0.0f, lsum = 0.0f;
+        for (int j0 = 0; j0 < ncc; j0 += kMergeThreads) {
+            const int j = j0 + tid;
+            float wj = 0.0f;
+            if (j < ncc) {
+                const float* pp = part_of(j);
+                const float m = __ldcg(pp + g * 128 + q);
+                const float l = __ldcg(pp + g * 128 + g + q);
+                wj = (m == -INFINITY) ? 0.0f : fast_exp2(m - M);
+                lsum = fmaf(wj, l, lsum);
+            }
+            s_w[tid] = wj;
+            __syncthreads();
+            const int nj = ncc - j0 < kMergeThreads ? ncc - j0 : kMergeThreads;
+            for (int jj0 = 0; jj0 < nj; jj0 += kMergeBatch) {
+                float v[kMergeBatch];
+#pragma unroll
+                for (int k = 0; k < kMergeBatch; ++k)
+                    v[k] = (jj0 + k < nj) ? __ldcg(part_of(j0 + jj0 + k) + q * 128 + tid) : 0.0f;
+#pragma unroll
+                for (int k = 0; k < kMergeBatch; ++k)
+                    if (jj0 + k < nj) acc = fmaf(s_w[jj0 + k], v[k], acc);
+            }
+            __syncthreads();                               // s_w is reused
+        }
+        const float L = merge_block_sum(lsum, s_red, warp, lane);
+        p.out[((int64_t)u.b * p.Hq + (int64_t)u.h * g + q) * 128 + tid] = L > 0.0f ? acc / L : 0.0f;
     }
 }
 
@@ -907,16 +1191,24 @@ template <int NT>
 cudaError_t launch_tc(const Params& p, int grid, cudaStream_t stream) {
     auto kern = decode_attention_tc_kernel<NT>;
     const int smem = (int)sizeof(Smem<NT>) + 1024;   // + alignment slack
-    static int configured_device = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_device != dev) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        configured_device = dev;
-    }
+    static int configured[kMaxDevices] = {};
+    cudaError_t e0 = ensure_smem_attribute(reinterpret_cast<const void*>(kern), smem, configured);
+    if (e0 != cudaSuccess) return e0;
     kern<<<grid, kThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // the merge grid, launched as a programmatic dependent of the attention grid
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kMergeThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, merge_split_units_kernel, p, grid);
 }
 
 }  // namespace

@@ -79,6 +79,64 @@ __device__ __forceinline__ uint32_t e2m1_from_float(float y) {
 }
 
 // ---------------------------------------------------------------------------
+// NVFP4 quantization of one 16-element micro-block (append path; also used by
+// the fused append + attention kernel)
+// ---------------------------------------------------------------------------
+template <bool F32>
+__device__ __forceinline__ void load16(const void* x, int64_t elem, float (&v)[16]) {
+    if (F32) {
+        const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + elem);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 f = __ldg(p + j);
+            v[4 * j + 0] = f.x;
+            v[4 * j + 1] = f.y;
+            v[4 * j + 2] = f.z;
+            v[4 * j + 3] = f.w;
+        }
+    } else {
+        const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(x) + elem);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const uint4 w = __ldg(p + j);
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                v[8 * j + 2 * k + 0] = __uint_as_float(ws[k] << 16);          // bf16 -> fp32, exact
+                v[8 * j + 2 * k + 1] = __uint_as_float(ws[k] & 0xFFFF0000u);
+            }
+        }
+    }
+}
+
+// Quantize one micro-block: returns the scale byte, writes 8 packed bytes.
+__device__ __forceinline__ uint32_t quantize_block(const float (&v)[16], float s_tensor, uint2& packed) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const float d6 = __fmul_rn(6.0f, s_tensor);
+    const float r = __fdiv_rn(amax, d6);
+    const uint32_t sb = e4m3_from_float(r);
+    const float den = __fmul_rn(e4m3_to_float(sb), s_tensor);
+    uint32_t c[16];
+    if (den == 0.0f) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) c[i] = (__float_as_uint(v[i]) >> 28) & 0x8u;
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) c[i] = e2m1_from_float(__fdiv_rn(v[i], den));
+    }
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        lo |= c[i] << (4 * i);
+        hi |= c[8 + i] << (4 * i);
+    }
+    packed = make_uint2(lo, hi);
+    return sb;
+}
+
+// ---------------------------------------------------------------------------
 // NVFP4 -> FP8 lookup
 // ---------------------------------------------------------------------------
 // The FP8 value of a code depends only on its 3-bit magnitude, the block's
@@ -86,20 +144,18 @@ __device__ __forceinline__ uint32_t e2m1_from_float(float y) {
 // A block's 8 values fit two 32-bit words (byte m = magnitude m), which
 // `byte_perm` then indexes with four 3-bit selectors at a time.
 // |c| * value(sb) has at most 6 significant bits, so the first product is
-// exact; the second is one fp32 rounding; the E4M3 conversion rounds to
-// nearest even and saturates at 448.
+// exact; the second is one fp32 rounding; the E4M3 conversion (the software
+// one above, nearest even, saturating at 448) is the one the quantizer uses
+// for its scale bytes, so the table needs no hardware conversion.
 __device__ __forceinline__ uint2 lut_words(uint32_t sb, float s_tensor) {
     if ((sb & 0x7Fu) == 0x7Fu) return make_uint2(0u, 0u);   // never written by quantize
     const float v = e4m3_to_float(sb & 0x7Fu);
-    float f[8];
+    uint32_t b[8];
 #pragma unroll
-    for (int m = 0; m < 8; ++m) f[m] = __fmul_rn(__fmul_rn(e2m1_magnitude((uint32_t)m), v), s_tensor);
-    uint16_t b01, b23, b45, b67;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(b01) : "f"(f[1]), "f"(f[0]));
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(b23) : "f"(f[3]), "f"(f[2]));
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(b45) : "f"(f[5]), "f"(f[4]));
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(b67) : "f"(f[7]), "f"(f[6]));
-    return make_uint2((uint32_t)b01 | ((uint32_t)b23 << 16), (uint32_t)b45 | ((uint32_t)b67 << 16));
+    for (int m = 0; m < 8; ++m)
+        b[m] = e4m3_from_float(__fmul_rn(__fmul_rn(e2m1_magnitude((uint32_t)m), v), s_tensor));
+    return make_uint2(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24),
+                      b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24));
 }
 
 // Dequantize 8 packed codes (one 32-bit word; element k in nibble k) to 8 FP8

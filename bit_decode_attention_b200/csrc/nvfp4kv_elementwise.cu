@@ -94,60 +94,6 @@ cudaError_t launch_calib(const void* x, bool f32, int64_t n, float* d_s_tensor, 
 // ordered (b, h, t, block) so that code and scale writes are contiguous in
 // the [B][H_kv][S_max][...] planes.
 // ---------------------------------------------------------------------------
-template <bool F32>
-__device__ __forceinline__ void load16(const void* x, int64_t elem, float (&v)[16]) {
-    if (F32) {
-        const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + elem);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float4 f = __ldg(p + j);
-            v[4 * j + 0] = f.x;
-            v[4 * j + 1] = f.y;
-            v[4 * j + 2] = f.z;
-            v[4 * j + 3] = f.w;
-        }
-    } else {
-        const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(x) + elem);
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const uint4 w = __ldg(p + j);
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                v[8 * j + 2 * k + 0] = __uint_as_float(ws[k] << 16);          // bf16 -> fp32, exact
-                v[8 * j + 2 * k + 1] = __uint_as_float(ws[k] & 0xFFFF0000u);
-            }
-        }
-    }
-}
-
-// Quantize one micro-block: returns the scale byte, writes 8 packed bytes.
-__device__ __forceinline__ uint32_t quantize_block(const float (&v)[16], float s_tensor, uint2& packed) {
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    const float d6 = __fmul_rn(6.0f, s_tensor);
-    const float r = __fdiv_rn(amax, d6);
-    const uint32_t sb = e4m3_from_float(r);
-    const float den = __fmul_rn(e4m3_to_float(sb), s_tensor);
-    uint32_t c[16];
-    if (den == 0.0f) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) c[i] = (__float_as_uint(v[i]) >> 28) & 0x8u;
-    } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) c[i] = e2m1_from_float(__fdiv_rn(v[i], den));
-    }
-    uint32_t lo = 0, hi = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        lo |= c[i] << (4 * i);
-        hi |= c[8 + i] << (4 * i);
-    }
-    packed = make_uint2(lo, hi);
-    return sb;
-}
-
 // Quantize-append of one plane (a1-a4); `item` enumerates (b, t, h, blk)
 // with blk fastest.  Index math in 32 bits when the item count fits.
 template <bool F32, typename I>

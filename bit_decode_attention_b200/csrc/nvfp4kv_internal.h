@@ -19,7 +19,19 @@ constexpr int kMaxBatchPerLaunch = 512;
 constexpr int kCtasPerSm = 2;
 constexpr int kMaxCtasPerSm = 3;
 
-int device_sm_count();  // multiprocessor count of the current device (cached)
+int device_sm_count();  // multiprocessor count of the current device (cached per device)
+
+// Host-side argument checks of nvfp4_decode_attention (planes, shapes,
+// pointers, alignment, dtype, softmax scale), without the workspace.
+nvfp4_status attention_precheck(const void* q, nvfp4_dtype q_dtype, int H_q, const nvfp4_kv_plane* k,
+                                const nvfp4_kv_plane* v, const float* d_s_tensor_k,
+                                const float* d_s_tensor_v, const int32_t* d_seq_lens,
+                                float softmax_scale, const float* out);
+
+// cudaFuncSetAttribute(kernel, MaxDynamicSharedMemorySize, bytes) once per
+// (kernel, device); `done` is the kernel's per-device flag array
+cudaError_t ensure_smem_attribute(const void* kernel, int bytes, int* done_flags);
+constexpr int kMaxDevices = 64;
 
 // floats per split-K partial slot: O [g][D], m [g], l [g], padded to a whole
 // float4 so that every slot starts 16-byte aligned
@@ -69,6 +81,16 @@ struct AttnLaunch {
     // paged cache: nullptr for contiguous planes (then S_max is the capacity)
     const int32_t* block_table;
     int page_tokens, max_pages, num_pages;
+    uint32_t wait_polls;  // give-up limit of the tensor-core kernel's pipeline waits
+    // append + attention (contiguous planes): start_pos != nullptr attends
+    // start_pos[b] + 1 tokens after appending one new token per sequence from
+    // x_k_new / x_v_new [B][1][Hkv][D] (fp32 when x_f32, else bf16) at slot
+    // start_pos[b]; new_lens (optional) receives start_pos[b] + 1
+    const int32_t* start_pos;
+    int32_t* new_lens;
+    const void* x_k_new;
+    const void* x_v_new;
+    bool x_f32;
 };
 
 cudaError_t launch_decode_attention(const AttnLaunch& a, cudaStream_t stream);

@@ -51,7 +51,11 @@ extern "C" nvfp4_status nvfp4_decode_attention_noalloc(
     const void* q, nvfp4_dtype q_dtype, int H_q, const nvfp4_kv_plane* k, const nvfp4_kv_plane* v,
     const float* d_s_tensor_k, const float* d_s_tensor_v, const int32_t* d_seq_lens,
     float softmax_scale, float* out, int32_t* d_status, nvfp4_stream_t stream) {
-    if (k == nullptr || v == nullptr) return NVFP4_ERR_INVALID_ARG;
+    // the same host checks as nvfp4_decode_attention, before anything is queued
+    const nvfp4_status pre = nvfp4kv::attention_precheck(q, q_dtype, H_q, k, v, d_s_tensor_k, d_s_tensor_v,
+                                                          d_seq_lens, softmax_scale, out);
+    if (pre != NVFP4_OK) return pre;
+    if (k->B == 0) return NVFP4_OK;
     const size_t need = nvfp4_decode_attention_workspace(k->B, H_q, k->H_kv, k->D);
     if (need == 0) return NVFP4_ERR_INVALID_ARG;
     if (need > kNoAllocScratchBytes) return NVFP4_ERR_WORKSPACE;   // shape too large for the buffer

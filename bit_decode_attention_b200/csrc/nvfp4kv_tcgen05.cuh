@@ -65,6 +65,17 @@ __device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t* r) {
         "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
 }
+__device__ __forceinline__ void tmem_st_x4(uint32_t taddr, const uint32_t* r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld_x4(uint32_t taddr, uint32_t* r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr)
+                 : "memory");
+}
 __device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, uint32_t* r) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
@@ -131,6 +142,54 @@ __device__ __forceinline__ void mma_e4m3_ss(uint32_t d_tmem, uint64_t a_desc, ui
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
         : "memory");
 }
+// Four MMAs accumulating into one D and the commit that signals their
+// completion, in one instruction sequence (separate asm statements per MMA
+// cost several times more issue cycles: each moves its operands into uniform
+// registers on its own).  D(tmem) (+)= A_k(tmem) * B_k(smem) for k = 0..3,
+// A_k at column a + 8k (K = 32 FP8 bytes each), B_k = b[k]; the first MMA
+// accumulates only when `acc` is non-zero; then one arrive on `bar` when all
+// MMAs this thread issued so far have completed.
+__device__ __forceinline__ void mma4_ts_commit(uint32_t d, uint32_t a, const uint64_t (&b)[4], uint32_t idesc,
+                                               uint32_t acc, uint64_t* bar) {
+    asm volatile(
+        "{\n\t.reg .pred p0, p1;\n\t"
+        "setp.ne.b32 p0, %9, 0;\n\t"
+        "setp.eq.b32 p1, %9, %9;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %5, %10, p0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%2], %6, %10, p1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%3], %7, %10, p1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%4], %8, %10, p1;\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%11];\n\t}"
+        ::"r"(d), "r"(a), "r"(a + 8), "r"(a + 16), "r"(a + 24), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]),
+          "r"(acc), "r"(idesc), "r"(smem_addr(bar))
+        : "memory");
+}
+// The same with A from shared memory: D(tmem) (+)= A_k(smem) * B_k(smem).
+__device__ __forceinline__ void mma4_ss_commit(uint32_t d, const uint64_t (&a)[4], const uint64_t (&b)[4],
+                                               uint32_t idesc, uint32_t acc, uint64_t* bar) {
+    asm volatile(
+        "{\n\t.reg .pred p0, p1;\n\t"
+        "setp.ne.b32 p0, %9, 0;\n\t"
+        "setp.eq.b32 p1, %9, %9;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %5, %10, p0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %2, %6, %10, p1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %3, %7, %10, p1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %4, %8, %10, p1;\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%11];\n\t}"
+        ::"r"(d), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]),
+          "r"(acc), "r"(idesc), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// One lane of the (converged) warp: true in exactly one lane.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // Arrive once on the mbarrier when every MMA this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* mbar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(

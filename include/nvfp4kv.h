@@ -125,6 +125,17 @@ const char* nvfp4_status_string(int status);
 /* Library version string (static). */
 const char* nvfp4_version(void);
 
+/* Testing hook for the failure path of the tensor-core attention kernel
+ * (head_dim 128, bf16 queries).  Its pipeline waits (one role waiting for
+ * another through a shared-memory barrier) give up after `polls` sleeping
+ * polls of up to 20 us each: the kernel then reports NVFP4_ERR_TIMEOUT
+ * through *d_status, skips its remaining work, waits (bounded) for the copies
+ * and MMAs it has issued, releases its tensor memory and returns.  polls = 0
+ * gives up at once unless the awaited phase has already completed; polls < 0
+ * restores the default (65536).  Applies to later calls from every thread.
+ * Host-only; needs no GPU. */
+void nvfp4_set_wait_limit(int64_t polls);
+
 /* Bytes of ONE plane (codes + scales) for the given shape: B * H_kv * S_max *
  * (D/2 + D/16).  Per element that is 4 code bits plus 8/16 scale bits = 4.5
  * bits, the format behind the memory table in [NVFP4-KV] "メモリ削減効果"
@@ -248,6 +259,35 @@ nvfp4_status nvfp4_decode_attention(const void* q, nvfp4_dtype q_dtype, int H_q,
                                     const int32_t* d_seq_lens, float softmax_scale,
                                     float* out, void* workspace, size_t workspace_bytes,
                                     int32_t* d_status, nvfp4_stream_t stream);
+
+/* Append one decode token per sequence, then attend over the cache including
+ * it, in one call ([NVFP4-KV] "量子化・逆量子化フロー": the new K/V are
+ * quantized to NVFP4 as they enter the cache, then FP8 attention runs over
+ * the dequantized cache).  Equivalent to nvfp4_kv_quantize_append_kv with
+ * n_new = 1 followed by nvfp4_decode_attention with seq_lens = start + 1, and
+ * bit-identical to that pair: same codes, scale bytes and output.  On the
+ * tensor-core path (head_dim 128, bf16 queries) it is ONE kernel launch (plus
+ * the split-K merge): the CTA whose range holds a sequence's last tile
+ * quantizes that sequence's new token before it loads the tile; other shapes
+ * run the append kernel first.
+ *   x_k_new, x_v_new  device [B][1][H_kv][D] of x_dtype, 16-byte aligned
+ *   d_start_pos       device int32 [B]: the new token goes to slot start_pos[b]
+ *                     and the attention covers start_pos[b] + 1 tokens
+ *   d_new_lens        device int32 [B] or NULL: receives start_pos[b] + 1; must
+ *                     not alias d_start_pos
+ *   every other argument as for nvfp4_decode_attention (seq_lens excepted)
+ * A sequence with start_pos < 0 or start_pos + 1 > S_max is not appended;
+ * NVFP4_ERR_CAPACITY goes to *d_status and its attention length is clamped
+ * to [0, S_max].  A non-finite or non-positive tensor scale skips the append
+ * with NVFP4_ERR_NONFINITE. */
+nvfp4_status nvfp4_decode_attention_append(const void* q, nvfp4_dtype q_dtype, int H_q,
+                                           const void* x_k_new, const void* x_v_new, nvfp4_dtype x_dtype,
+                                           const int32_t* d_start_pos, int32_t* d_new_lens,
+                                           const nvfp4_kv_plane* k, const nvfp4_kv_plane* v,
+                                           const float* d_s_tensor_k, const float* d_s_tensor_v,
+                                           float softmax_scale, float* out, void* workspace,
+                                           size_t workspace_bytes, int32_t* d_status,
+                                           nvfp4_stream_t stream);
 
 /* nvfp4_decode_attention over paged K and V planes.  k and v share one block
  * table (the same pointer) and agree in B, H_kv, page_tokens, max_pages, D;

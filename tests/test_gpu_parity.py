@@ -485,3 +485,115 @@ def test_paged_bad_table_entries_are_reported(nv):
     torch.cuda.synchronize()
     assert status.item() == nv.NVFP4_ERR_INVALID_ARG
     assert torch.isfinite(out).all()
+
+
+def test_dequant_lookup_all_scale_bytes_many_tensor_scales(nv):
+    """The FP8 lookup every dequant path shares, against the oracle: every
+    (scale byte 0..126, code 0..15) pair -- one plane of 16 tokens x 8 blocks,
+    block j holding all 16 codes under scale byte 8t + j -- under 600 tensor
+    scales (log-uniform over 2^-40 .. 2^24, plus powers of two and values just
+    above and below them), covering normal, subnormal, zero and saturated FP8
+    results."""
+    S, D = 16, 128
+    codes = np.zeros((1, 1, S, D // 2), np.uint8)
+    scales = np.zeros((1, 1, S, D // 16), np.uint8)
+    nib = np.arange(16, dtype=np.uint8)
+    for t in range(S):
+        for j in range(D // 16):
+            scales[0, 0, t, j] = min(8 * t + j, 0x7E)
+            codes[0, 0, t, 8 * j:8 * j + 8] = nib[0::2] | (nib[1::2] << 4)
+    plane = nv.KVPlane(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda())
+    lens = np.array([S], np.int32)
+    lens_d = torch.from_numpy(lens).cuda()
+    rng = np.random.default_rng(5)
+    sts = list(np.exp2(rng.uniform(-40, 24, 560)).astype(np.float32))
+    for e in range(-30, 21, 5):
+        p = np.float32(2.0 ** e)
+        sts += [p, np.nextafter(p, np.float32(0)), np.nextafter(p, np.float32(np.inf)),
+                np.float32(p * 1.5)]
+    out = torch.empty(1, 1, S, D, dtype=torch.uint8, device="cuda")
+    for st in sts:
+        st = np.float32(st)
+        s = torch.tensor([st], dtype=torch.float32, device="cuda")
+        got = nv.nvfp4_kv_dequant_fp8(plane, s, lens_d, out=out).cpu().numpy()
+        want = oracle.dequant_planes(codes, scales, st, lens)
+        np.testing.assert_array_equal(got, want, err_msg="tensor scale %r" % float(st))
+
+
+# ---------------------------------------------------------------------------
+# append + attention in one call
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("D,q_dtype", [(128, "bf16"), (128, "f32"), (64, "bf16")])
+def test_append_attention_matches_two_calls_and_oracle(nv, D, q_dtype):
+    """nvfp4_decode_attention_append equals quantize_append_kv + decode
+    attention bit for bit (planes, new lengths, output), and the oracle within
+    tolerance; sequences with 0, 1, 127 (the new token opens a tile), 700 and
+    4100 cached tokens, and one whose slot is past the capacity."""
+    w = synthetic.shrink(synthetic.get("gqa"), B=6, Hq=16, Hkv=2, D=D)
+    lens = [700, 1, 127, 0, 4100, 50]
+    S_max = synthetic.capacity(4101)
+    c = Case(w, lens=lens, S_max=S_max, q_dtype=q_dtype)
+    start = list(lens)
+    start[5] = S_max                                      # past the capacity: not appended
+    start_d = torch.tensor(start, dtype=torch.int32, device="cuda")
+    xk = synthetic.kv_tokens(w, 1, "k", stream=9)
+    xv = synthetic.kv_tokens(w, 1, "v", stream=9)
+    xk_d, xv_d = to_dev(xk, w.dtype), to_dev(xv, w.dtype)
+    planes = {}
+    for key in ("two", "one"):
+        planes[key] = (nv.KVPlane(c.k.codes.clone(), c.k.scales.clone()),
+                       nv.KVPlane(c.v.codes.clone(), c.v.scales.clone()))
+    st_two = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st_one = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lens_two = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+    lens_one = torch.full((w.B,), -5, dtype=torch.int32, device="cuda")
+    k2, v2 = planes["two"]
+    nv.nvfp4_kv_quantize_append_kv(xk_d, xv_d, start_d, c.sk, c.sv, k2, v2, new_lens=lens_two, status=st_two)
+    att_lens = start_d + 1
+    want_dev = nv.nvfp4_decode_attention(c.q_dev, k2, v2, c.sk, c.sv, att_lens, status=st_two)
+    k1, v1 = planes["one"]
+    got = nv.nvfp4_decode_attention_append(c.q_dev, xk_d, xv_d, start_d, k1, v1, c.sk, c.sv,
+                                           new_lens=lens_one, status=st_one)
+    torch.cuda.synchronize()
+    assert st_two.item() == nv.NVFP4_ERR_CAPACITY and st_one.item() == nv.NVFP4_ERR_CAPACITY
+    assert torch.equal(k1.codes, k2.codes) and torch.equal(k1.scales, k2.scales)
+    assert torch.equal(v1.codes, v2.codes) and torch.equal(v1.scales, v2.scales)
+    assert lens_one.tolist()[:5] == lens_two.tolist()[:5] == [s + 1 for s in start[:5]]
+    assert torch.equal(got, want_dev)
+    # oracle: the prefill planes, the new token at slot start, fp64 attention over start + 1
+    got = got.cpu().numpy()
+    for b in range(5):
+        kc, ks, vc, vs = c.oracle_planes(b)
+        at = np.array([start[b]], np.int32)
+        assert oracle.quantize_append(xk[b:b + 1].numpy(), at, c.sk_o, kc, ks) == 0
+        assert oracle.quantize_append(xv[b:b + 1].numpy(), at, c.sv_o, vc, vs) == 0
+        want = oracle.decode_attention_nvfp4(c.q[b:b + 1].numpy(), kc, ks, vc, vs, c.sk_o, c.sv_o,
+                                             np.array([start[b] + 1], np.int32))
+        assert_attention_close(got[b:b + 1], want)
+
+
+# ---------------------------------------------------------------------------
+# failure path: a pipeline wait that gives up
+# ---------------------------------------------------------------------------
+def test_attention_wait_timeout_reports_and_recovers(nv):
+    """With a zero wait limit the tensor-core kernel's first wait that is not
+    already complete gives up: the call reports NVFP4_ERR_TIMEOUT through the
+    status word, drains its copies and MMAs, releases tensor memory and
+    returns (no hang, no fault), and the next call with the default limit is
+    correct again.  The limit is set on the host; nothing on the device is
+    made to fail."""
+    c = Case(synthetic.shrink(synthetic.get("long64k"), L=3000, Hq=16, Hkv=2))
+    want = c.oracle_attention()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    try:
+        nv.nvfp4_set_wait_limit(0)
+        nv.nvfp4_decode_attention(c.q_dev, c.k, c.v, c.sk, c.sv, c.seq_lens, status=status)
+        torch.cuda.synchronize()
+    finally:
+        nv.nvfp4_set_wait_limit(-1)
+    assert status.item() == nv.NVFP4_ERR_TIMEOUT
+    status.zero_()
+    got = nv.nvfp4_decode_attention(c.q_dev, c.k, c.v, c.sk, c.sv, c.seq_lens, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert_attention_close(got.cpu().numpy(), want)
