@@ -67,14 +67,17 @@ constexpr int NTERM = 3;                              // E4M3 terms of P
 //   warps  0- 3  K dequant, head_dim  0-63      warps 16-19  V dequant, head_dim 64-127
 //   warps  4- 7  softmax group 0 (queries 0 .. NQ/2-1)
 //   warps  8-11  K dequant, head_dim 64-127     warps 20-23  softmax group 1 (NQ/2 .. NQ-1)
-//   warps 12-15  V dequant, head_dim  0-63      warp 24 loads, warp 25 MMAs (26-27 idle)
+//   warps 12-15  V dequant, head_dim  0-63      warp 24 loads, 25 Q.K^T MMAs, 26 P.V MMAs,
+//                                               27 the fused append's new tokens
 constexpr int kS0Warp0 = 4;
 constexpr int kK1Warp0 = 8;
 constexpr int kV0Warp0 = 12;
 constexpr int kV1Warp0 = 16;
 constexpr int kS1Warp0 = 20;
 constexpr int kLoadWarp = 24;
-constexpr int kMmaWarp = 25;
+constexpr int kMmaWarp = 25;                          // Q.K^T
+constexpr int kPvWarp = 26;                           // P.V
+constexpr int kAppendWarp = 27;                       // new tokens of the fused append
 constexpr int kThreads = 28 * 32;
 // registers per thread after the prologue (setmaxnreg); the launch holds
 // kThreads x 72, and 128 x (2 x 112 + 4 x 56 + 56) = 64,512 of them
@@ -111,9 +114,11 @@ struct __align__(1024) Smem {
     uint64_t vfull[kBuf], pfull[kBuf], pvdone[kBuf];
     uint64_t qfull[2];
     uint64_t mma_done;
+    uint64_t appended;                                // the fused append's new tokens are written
     int32_t lens[kMaxBatchPerLaunch];
     int32_t prefix[kMaxBatchPerLaunch + 1];
     float cscale[2][C::NQ];
+    alignas(16) uint8_t qraw[2][128][16];             // next unit's query loads, per softmax thread
     float red[4][C::NQ];
     int32_t warp_tot[kThreads / 32];
     int32_t warp_empty[kThreads / 32];
@@ -286,6 +291,29 @@ __device__ __forceinline__ void fetch_q(const Params& p, int b, int h, int q0, i
     }
 }
 
+// The same loads as fetch_q, but asynchronous into this thread's 16-byte slot
+// of shared memory (rows past the group are zero-filled), so that no register
+// holds them while the segment runs; take_q waits for them and reads them.
+template <int NT>
+__device__ __forceinline__ void fetch_q_async(const Params& p, int b, int h, int q0, int t, uint8_t* slot) {
+    constexpr int PER = QRaw<NT>::PER;
+    constexpr int TPQ = 128 / PER;
+    const int q = q0 + t / TPQ;
+    const int d0 = (t % TPQ) * PER;
+    const bool valid = q < p.g;
+    const int64_t row = ((int64_t)b * p.Hq + (int64_t)h * p.g + (valid ? q : 0)) * 128 + d0;
+    const uint16_t* src = reinterpret_cast<const uint16_t*>(p.q) + row;
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2, %3;\n\tcp.async.commit_group;" ::"r"(smem_u32(slot)),
+                 "l"(src), "n"(PER * 2), "r"(valid ? PER * 2 : 0)
+                 : "memory");
+}
+template <int NT>
+__device__ __forceinline__ void take_q(const uint8_t* slot, QRaw<NT>& raw) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+#pragma unroll
+    for (int k = 0; k < QRaw<NT>::PER / 2; ++k) raw.w[k] = reinterpret_cast<const uint32_t*>(slot)[k];
+}
+
 template <int NT>
 __device__ __forceinline__ void build_q(const Params& p, uint8_t* qb, float* cscale, const QRaw<NT>& raw,
                                         int q0, int t) {
@@ -388,29 +416,31 @@ struct TileWalker {
 };
 
 // ---------------------------------------------------------------------------
-// Fused append (a2-a4 for one token): every unit whose last tile lies in
-// [t_begin, t_end) gets its new token -- K and V, 8 blocks each, one lane per
-// block (lanes 0-7 K, 8-15 V) of warp (unit ordinal % warps) -- quantized with
-// the same block quantizer as nvfp4_kv_quantize_append and written at slot
-// start_pos[b].  A sequence whose slot is out of range is skipped (the
-// prologue reported it); a non-finite or non-positive tensor scale skips
-// everything with NVFP4_ERR_NONFINITE.  The writers then order their global
-// stores before the async proxy's bulk copies (the caller's CTA barrier
-// follows).
+// Fused append (a2-a4 for one token), by one warp: every unit whose last tile
+// lies in [t_begin, t_end) gets its new token -- K and V, 8 blocks each, one
+// lane per block (half-warp h of the warp takes every second such unit; lanes
+// 0-7 of a half K, 8-15 V) -- quantized with the same block quantizer as
+// nvfp4_kv_quantize_append and written at slot start_pos[b].  A sequence whose
+// slot is out of range is skipped (the prologue reported it); a non-finite or
+// non-positive tensor scale skips everything with NVFP4_ERR_NONFINITE.  Every
+// writer then orders its global stores before later async-proxy reads (the
+// load warp's bulk copies, after the caller's barrier arrive).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void append_new_tokens(const Params& p, const int32_t* prefix, const int32_t* lens,
-                                               int B, int64_t t_begin, int64_t t_end, float st_k,
-                                               float st_v, int warp, int lane) {
+                                                  int B, int64_t t_begin, int64_t t_end, float st_k,
+                                                  float st_v, int lane) {
     const bool ok_k = st_k > 0.0f && st_k <= 3.4028234663852886e38f;
     const bool ok_v = st_v > 0.0f && st_v <= 3.4028234663852886e38f;
+    if (!(ok_k && ok_v) && lane == 0) report(p.status, NVFP4_ERR_NONFINITE);
+    const int half = lane >> 4;
+    const bool is_v = (lane & 15) >= 8;
+    const int blk = lane & 7;
     int ui = 0;
     for (int64_t seg_lo = t_begin; seg_lo < t_end;) {
         const Unit u = find_unit<TILE>(prefix, lens, B, p.Hkv, seg_lo);
         if (u.U1 <= t_end) {
-            if (ui % (kThreads / 32) == warp && lane < 16) {
+            if ((ui & 1) == half) {
                 const int start = p.start_pos[u.b];
-                const bool is_v = lane >= 8;
-                const int blk = lane & 7;
                 const bool in_range = start >= 0 && start + 1 <= p.S_max;
                 if (in_range && (is_v ? ok_v : ok_k)) {
                     float v[16];
@@ -426,7 +456,6 @@ __device__ __forceinline__ void append_new_tokens(const Params& p, const int32_t
                     scales[slot * 8 + blk] = (uint8_t)sb;
                     if (!is_v && blk == 0 && u.h == 0 && p.new_lens != nullptr) p.new_lens[u.b] = start + 1;
                 }
-                if (!(ok_k && ok_v) && lane == 0) report(p.status, NVFP4_ERR_NONFINITE);
             }
             ++ui;
         }
@@ -518,6 +547,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
         if (lane == 0) sm.warp_empty[warp] = empty;
     }
 
+    // softmax groups with real queries: the second group (queries NQ/2 ..)
+    // has none when the GQA group fits the first one's
+    const int n_sgrp = p.g > NQ / 2 ? 2 : 1;
+
     // ---- tensor memory, barriers, lookup tables, zeroed P buffers ----
     if (warp == kMmaWarp) {
         tc::tmem_alloc(&sm.tmem_base, C::kTmemCols);
@@ -527,6 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
     TileWalker load_walk;
     load_walk.start(t_begin, t_end);
     uint32_t load_w = 0;
+    bool load_pending = false;                        // the walker's current tile is not issued yet
     if (warp == kLoadWarp && lane == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.full[s], 1);
@@ -535,19 +569,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
         for (int b = 0; b < kBuf; ++b) {
             mbar_init(&sm.kfull[b], 8);
             mbar_init(&sm.qkdone[b], 1);
-            mbar_init(&sm.sempty[b], 8);
+            mbar_init(&sm.sempty[b], 4 * n_sgrp);
             mbar_init(&sm.vfull[b], 8);
-            mbar_init(&sm.pfull[b], 8);
+            mbar_init(&sm.pfull[b], 4 * n_sgrp);
             mbar_init(&sm.pvdone[b], 1);
         }
-        mbar_init(&sm.qfull[0], 8);
-        mbar_init(&sm.qfull[1], 8);
-        mbar_init(&sm.mma_done, 1);
+        mbar_init(&sm.qfull[0], 4 * n_sgrp);
+        mbar_init(&sm.qfull[1], 4 * n_sgrp);
+        mbar_init(&sm.mma_done, 2);                   // both MMA warps commit
+        mbar_init(&sm.appended, 1);
         fence_mbar_init();
         sm.abort_flag = 0;
-        // the first two tiles only: the CTA barrier below waits for this lane
-        // (in the fused append mode every copy waits for the new tokens)
-        while (p.x_k_new == nullptr && load_w < 2u && load_walk.next(sm.prefix, sm.lens, B, p.Hkv)) {
+        // the first two tiles only: the CTA barrier below waits for this lane;
+        // in the fused append mode a unit's last tile (it holds the new token)
+        // waits for the append warp
+        while (load_w < 2u && load_walk.next(sm.prefix, sm.lens, B, p.Hkv)) {
+            if (p.x_k_new != nullptr && load_walk.last == load_walk.u.U1 - 1) {
+                load_pending = true;
+                break;
+            }
             issue_tile<128, TILE>(p, load_walk.u, load_walk.last, sm.ring[load_w], &sm.full[load_w]);
             ++load_w;
         }
@@ -556,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
     const int wg = warp >> 2;                          // warpgroup
     const bool is_softmax = wg == kS0Warp0 / 4 || wg == kS1Warp0 / 4;
     const int sgrp = wg == kS1Warp0 / 4 ? 1 : 0;       // softmax group
-    if (is_softmax) {
+    if (is_softmax && sgrp < n_sgrp) {
         const Unit u0 = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, t_begin);
         fetch_q<NT>(p, u0.b, u0.h, sgrp * (NQ / 2), 32 * (warp & 3) + lane, q_first);
     }
@@ -579,12 +619,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    if (p.x_k_new != nullptr) {
-        // fused append: the CTA that owns a unit's last tile quantizes the
-        // unit's new token (slot L - 1) before any copy of that tile is issued
-        append_new_tokens(p, sm.prefix, sm.lens, B, t_begin, t_end, st_k, st_v, warp, lane);
-        __syncthreads();
-    }
     const uint32_t tbase = sm.tmem_base;
     int32_t* const abort_flag = &sm.abort_flag;
     launch_dependents();                              // the merge grid may be scheduled now
@@ -601,11 +635,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
         // ================= bulk copies into the ring =================
         if (lane == 0) {
             uint32_t w = load_w;                       // the first stages went out in the prologue
-            while (load_walk.next(sm.prefix, sm.lens, B, p.Hkv)) {
+            bool appended = p.x_k_new == nullptr;
+            while (load_pending || load_walk.next(sm.prefix, sm.lens, B, p.Hkv)) {
+                load_pending = false;
                 const int s = (int)(w % kStages);
                 if (w >= (uint32_t)kStages &&
                     !wait_one(&sm.empty[s], ((w / kStages) - 1) & 1u, abort_flag, p.status, polls))
                     break;
+                if (!appended && load_walk.last == load_walk.u.U1 - 1) {
+                    if (!wait_one(&sm.appended, 0, abort_flag, p.status, polls)) break;
+                    appended = true;
+                }
                 issue_tile<128, TILE>(p, load_walk.u, load_walk.last, sm.ring[s], &sm.full[s]);
                 ++w;
             }
@@ -618,82 +658,84 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
                 }
             }
         }
-    } else if (warp == kMmaWarp) {
+    } else if (warp == kMmaWarp || warp == kPvWarp) {
         // ================= tensor-core MMAs =================
-        // The whole warp runs the schedule and its waits (every value stays
+        // Two issuing warps, so that neither product waits behind the other:
+        // warp kMmaWarp issues Q.K^T as soon as a tile's K is in tensor
+        // memory, warp kPvWarp issues P.V as soon as its P and V^T are in
+        // shared memory (a commit tracks the issuing thread's own MMAs).  The
+        // whole warp runs the schedule and its waits (every value stays
         // warp-uniform); one elected lane issues each group of four MMAs
         // together with its commit.
-        const uint32_t idesc_qk = tc::idesc_e4m3(128, NS, false, false, false);
-        const uint32_t idesc_pv = tc::idesc_e4m3(128, C::NP, true, true, false);
-        // descriptors of buffer 0; buffer b and k-step ks add to the
-        // start-address field (16-byte units, no carry out of its 14 bits)
-        const uint64_t qdesc0 = tc::smem_desc(tc::smem_addr(sm.qb[0]), 128, 1024);
-        const uint64_t vdesc0 = tc::smem_desc(tc::smem_addr(sm.vt[0]), 128, 2048);
-        const uint64_t pdesc0 = tc::smem_desc(tc::smem_addr(sm.pb[0]), 128, 2048);
-        constexpr uint64_t kQStep = (C::NS * 128) >> 4, kVStep = (128 * TILE) >> 4,
-                           kPStep = (C::NP * TILE) >> 4;
         TileWalker walk;
         walk.start(t_begin, t_end);
         bool ok = true;
-        int32_t q_seg = -1;                            // segment whose query operand is in place
-        // Q.K^T of tile wq: S(b) = K(b) . Q'^T, then commit to qkdone[b]
-        auto issue_qk = [&](uint32_t wq, int32_t jq) -> bool {
-            const int b = (int)(wq % kBuf);
-            const uint32_t ph = (wq / kBuf) & 1u;
-            if (q_seg != jq) {
-                if (!wait_warp(&sm.qfull[jq & 1], ((uint32_t)jq >> 1) & 1u, abort_flag, p.status, polls))
-                    return false;
-                q_seg = jq;
+        if (warp == kMmaWarp) {
+            const uint32_t idesc_qk = tc::idesc_e4m3(128, NS, false, false, false);
+            // descriptor of buffer 0; buffer and k-step add to the start-address
+            // field (16-byte units, no carry out of its 14 bits)
+            const uint64_t qdesc0 = tc::smem_desc(tc::smem_addr(sm.qb[0]), 128, 1024);
+            constexpr uint64_t kQStep = (C::NS * 128) >> 4;
+            int32_t q_seg = -1;                        // segment whose query operand is in place
+            // Q.K^T of tile w: S(b) = K(b) . Q'^T, then commit to qkdone[b]
+            for (uint32_t w = 0; ok && walk.next(sm.prefix, sm.lens, B, p.Hkv); ++w) {
+                const int32_t jq = walk.j;
+                const int b = (int)(w % kBuf);
+                const uint32_t ph = (w / kBuf) & 1u;
+                if (q_seg != jq) {
+                    ok = wait_warp(&sm.qfull[jq & 1], ((uint32_t)jq >> 1) & 1u, abort_flag, p.status, polls);
+                    q_seg = jq;
+                }
+                ok = ok && wait_warp(&sm.kfull[b], ph, abort_flag, p.status, polls);
+                ok = ok && (w < (uint32_t)kBuf || wait_warp(&sm.sempty[b], ph ^ 1u, abort_flag, p.status, polls));
+                if (!ok) break;
+                tc::fence_after_sync();
+                const uint64_t qd = qdesc0 + (uint64_t)(jq & 1) * kQStep;
+                const uint64_t bq[4] = {qd, qd + 16, qd + 32, qd + 48};
+                if (tc::elect_one())
+                    tc::mma4_ts_commit(tbase + C::COL_S + NS * b, tbase + C::COL_K + 32 * b, bq, idesc_qk, 0u,
+                                       &sm.qkdone[b]);
+                __syncwarp();
             }
-            if (!wait_warp(&sm.kfull[b], ph, abort_flag, p.status, polls)) return false;
-            if (wq >= (uint32_t)kBuf && !wait_warp(&sm.sempty[b], ph ^ 1u, abort_flag, p.status, polls))
-                return false;
-            tc::fence_after_sync();
-            const uint64_t qd = qdesc0 + (uint64_t)(jq & 1) * kQStep;
-            const uint64_t bq[4] = {qd, qd + 16, qd + 32, qd + 48};
-            if (tc::elect_one())
-                tc::mma4_ts_commit(tbase + C::COL_S + NS * b, tbase + C::COL_K + 32 * b, bq, idesc_qk, 0u,
-                                   &sm.qkdone[b]);
-            __syncwarp();
-            return true;
-        };
-        // P.V of tile wp: O += V^T(b) . P^T(b), then commit to pvdone[b]; O
-        // restarts with the first tile of each unit
-        auto issue_pv = [&](uint32_t wp, bool first) -> bool {
-            const int b = (int)(wp % kBuf);
-            const uint32_t ph = (wp / kBuf) & 1u;
-            if (!wait_warp(&sm.vfull[b], ph, abort_flag, p.status, polls)) return false;
-            if (!wait_warp(&sm.pfull[b], ph, abort_flag, p.status, polls)) return false;
-            tc::fence_after_sync();
-            const uint64_t vd = vdesc0 + (uint64_t)b * kVStep;
-            const uint64_t pd = pdesc0 + (uint64_t)b * kPStep;
-            const uint64_t av[4] = {vd, vd + 32, vd + 64, vd + 96};
-            const uint64_t bp[4] = {pd, pd + 32, pd + 64, pd + 96};
-            if (tc::elect_one())
-                tc::mma4_ss_commit(tbase + C::COL_O, av, bp, idesc_pv, first ? 0u : 1u, &sm.pvdone[b]);
-            __syncwarp();
-            return true;
-        };
-        bool have = walk.next(sm.prefix, sm.lens, B, p.Hkv);
-        if (have) ok = issue_qk(0, walk.j);
-        uint32_t w = 0;
-        while (ok && have) {
-            const bool first = walk.first;             // of tile w
-            have = walk.next(sm.prefix, sm.lens, B, p.Hkv);
-            if (have) ok = issue_qk(w + 1, walk.j);
-            if (ok) ok = issue_pv(w, first);
-            ++w;
+        } else {
+            const uint32_t idesc_pv = tc::idesc_e4m3(128, C::NP, true, true, false);
+            const uint64_t vdesc0 = tc::smem_desc(tc::smem_addr(sm.vt[0]), 128, 2048);
+            const uint64_t pdesc0 = tc::smem_desc(tc::smem_addr(sm.pb[0]), 128, 2048);
+            constexpr uint64_t kVStep = (128 * TILE) >> 4, kPStep = (C::NP * TILE) >> 4;
+            // P.V of tile w: O += V^T(b) . P^T(b), then commit to pvdone[b]; O
+            // restarts with the first tile of each unit
+            for (uint32_t w = 0; ok && walk.next(sm.prefix, sm.lens, B, p.Hkv); ++w) {
+                const int b = (int)(w % kBuf);
+                const uint32_t ph = (w / kBuf) & 1u;
+                ok = wait_warp(&sm.pfull[b], ph, abort_flag, p.status, polls) &&
+                     wait_warp(&sm.vfull[b], ph, abort_flag, p.status, polls);
+                if (!ok) break;
+                tc::fence_after_sync();
+                const uint64_t vd = vdesc0 + (uint64_t)b * kVStep;
+                const uint64_t pd = pdesc0 + (uint64_t)b * kPStep;
+                const uint64_t av[4] = {vd, vd + 32, vd + 64, vd + 96};
+                const uint64_t bp[4] = {pd, pd + 32, pd + 64, pd + 96};
+                if (tc::elect_one())
+                    tc::mma4_ss_commit(tbase + C::COL_O, av, bp, idesc_pv, walk.first ? 0u : 1u, &sm.pvdone[b]);
+                __syncwarp();
+            }
         }
         // every issued MMA must complete before tensor memory is released
         if (tc::elect_one()) tc::mma_commit(&sm.mma_done);
         __syncwarp();
         if (!mbar_wait_sleep(&sm.mma_done, 0, kWaitPolls)) report(p.status, NVFP4_ERR_TIMEOUT);
         __syncwarp();
+    } else if (warp == kAppendWarp) {
+        // ================= the fused append's new tokens =================
+        if (p.x_k_new != nullptr) {
+            append_new_tokens(p, sm.prefix, sm.lens, B, t_begin, t_end, st_k, st_v, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.appended);
+        }
     } else if (wg == 0 || wg == kK1Warp0 / 4) {
         // ======== K dequant: head_dim half h of token t's K row ========
-        // Software-pipelined: tile w's lookups, the publication of tile w - 1's
-        // tensor-memory stores, tile w + 1's raw data, then tile w's dequant
-        // and store -- each step's latency hides behind the next.
+        // Tile w + 1's raw data is read (and its ring stage released) before
+        // tile w's dequant, so that read's latency hides behind the dequant.
         regs_dec<kRegsDequant>();
         const int h = wg == 0 ? 0 : 1;                     // head_dim [64h, 64h + 64)
         const int t = 32 * (warp & 3) + lane;              // token, tensor-memory lane
@@ -722,12 +764,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
 #pragma unroll
             for (int i = 0; i < 4; ++i) l[i] = lut_k[((sk >> (8 * i)) & 0x7F) * kLutCopies];
             const uint4 c0 = xk[0], c1 = xk[1];
-            if (w >= 1) {                                  // tile w - 1 is in tensor memory
-                tc::tmem_wait_st();
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.kfull[(w - 1) % kBuf]);
-            }
             if (w + 1 < n_work) ok = fetch(w + 1);
             // Q.K^T of tile w - kBuf has read this K buffer
             if (!ok || (w >= kBuf && !wait_warp(&sm.qkdone[b], ph ^ 1u, abort_flag, p.status, polls))) {
@@ -745,17 +781,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
             dequant_word(c1.z, l[3].x, l[3].y, kf[12], kf[13]);
             dequant_word(c1.w, l[3].x, l[3].y, kf[14], kf[15]);
             tmem_st_x16(trow + C::COL_K + 32 * b + 16 * h, kf);
-        }
-        if (ok && n_work > 0) {
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.kfull[(n_work - 1) % kBuf]);
+            if (lane == 0) mbar_arrive(&sm.kfull[b]);     // Q.K^T of tile w may start
         }
     } else if (wg == kV0Warp0 / 4 || wg == kV1Warp0 / 4) {
         // ======== V dequant: head_dim half h of token t's V row -> V^T ========
-        // Pipelined like the K warps: tile w - 1's V^T stores are published
-        // (proxy fence, arrive) one step later, while tile w's lookups fly.
+        // Reads tile w + 1's raw data ahead, like the K warps.
         regs_dec<kRegsDequant>();
         const int h = wg == kV0Warp0 / 4 ? 0 : 1;
         const int t = 32 * (warp & 3) + lane;              // token
@@ -789,11 +822,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
                 l[2 * j + 1] = lut_v[((sv >> (16 * cc + 8)) & 0x7F) * kLutCopies];
             }
             const uint4 c[2] = {xv[0], xv[1]};
-            if (w >= 1) {                                  // tile w - 1's V^T is in shared memory
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.vfull[(w - 1) % kBuf]);
-            }
             if (w + 1 < n_work) ok = fetch(w + 1);
             // P.V of tile w - kBuf has read this V^T buffer
             if (!ok || (w >= kBuf && !wait_warp(&sm.pvdone[b], ph ^ 1u, abort_flag, p.status, polls))) {
@@ -813,12 +841,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
                 *reinterpret_cast<uint4*>(dst + (2 * cc) * 2048) = o0;
                 *reinterpret_cast<uint4*>(dst + (2 * cc + 1) * 2048) = o1;
             }
-        }
-        if (ok && n_work > 0) {
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.vfull[(n_work - 1) % kBuf]);
+            if (lane == 0) mbar_arrive(&sm.vfull[b]);     // P.V of tile w may start
         }
+    } else if (is_softmax && sgrp >= n_sgrp) {
+        // a group with padding queries only: nothing to do (its P columns stay
+        // the zeros of the prologue)
+        regs_inc<kRegsSoftmax>();
     } else if (is_softmax) {
         // ============ softmax, P, output: group sgrp owns queries q0 .. q0 + NH - 1 ============
         regs_inc<kRegsSoftmax>();
@@ -837,19 +867,45 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
             softmax_sync(bar_id);
             if (lane == 0) mbar_arrive(&sm.qfull[0]);
         }
+        // Each unit's query operand is built when the unit BEFORE it starts, so
+        // that Q.K^T of a unit's first tile never waits for the softmax of the
+        // previous unit's last tile (the pipeline does not drain at a unit
+        // boundary); its loads are issued one unit earlier still.
+        uint8_t* const qslot = sm.qraw[sgrp][t];
+        {
+            const Unit u0 = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, t_begin);
+            if (u0.U1 < t_end) {
+                const Unit u1 = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, u0.U1);
+                fetch_q_async<NT>(p, u1.b, u1.h, q0, t, qslot);
+            }
+        }
         for (int64_t seg_lo = t_begin; seg_lo < t_end; ++j) {
             const Unit u = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, seg_lo);
             const int64_t seg_hi = u.U1 < t_end ? u.U1 : t_end;
             const bool has_next = seg_hi < t_end;
-            QRaw<NT> qnext;
-            if (has_next) {                                // loads in flight during this segment
-                const Unit un = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, seg_hi);
-                fetch_q<NT>(p, un.b, un.h, q0, t, qnext);
-            }
             float cs[NH], m_run[NH], l_run[NH];
 #pragma unroll
+            for (int q = 0; q < NH; ++q) cs[q] = sm.cscale[j & 1u][q0 + q];
+            if (has_next) {
+                // query rows of the next unit; their buffer was last read by the
+                // Q.K^T MMAs of the unit before this one, all complete by now
+                // (this group has read every score of that unit)
+                {
+                    QRaw<NT> qnext;
+                    take_q<NT>(qslot, qnext);
+                    build_q<NT>(p, sm.qb[(j + 1) & 1u], sm.cscale[(j + 1) & 1u], qnext, q0, t);
+                }
+                fence_proxy_async_smem();
+                softmax_sync(bar_id);
+                if (lane == 0) mbar_arrive(&sm.qfull[(j + 1) & 1u]);
+                const Unit un = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, seg_hi);
+                if (un.U1 < t_end) {                       // loads for the unit after it
+                    const Unit un2 = find_unit<TILE>(sm.prefix, sm.lens, B, p.Hkv, un.U1);
+                    fetch_q_async<NT>(p, un2.b, un2.h, q0, t, qslot);
+                }
+            }
+#pragma unroll
             for (int q = 0; q < NH; ++q) {
-                cs[q] = sm.cscale[j & 1u][q0 + q];
                 m_run[q] = -INFINITY;
                 l_run[q] = 0.0f;
             }
@@ -966,14 +1022,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
             }
 
             // ---- segment end ----
-            if (has_next) {
-                // query rows of the next unit; their buffer was last read by the
-                // Q.K^T MMAs of the unit before this one, all complete by now
-                build_q<NT>(p, sm.qb[(j + 1) & 1u], sm.cscale[(j + 1) & 1u], qnext, q0, t);
-                fence_proxy_async_smem();
-                softmax_sync(bar_id);
-                if (lane == 0) mbar_arrive(&sm.qfull[(j + 1) & 1u]);
-            }
             float o[NH];
 #pragma unroll
             for (int q = 0; q < NH; ++q) o[q] = 0.0f;
@@ -1048,42 +1096,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
 // ---------------------------------------------------------------------------
 // Split-K merge of the units the attention grid left in partials:
 //     out = sum_j w_j O_j / sum_j w_j l_j,   w_j = 2^(m_j - M),  M = max_j m_j
-// over the contributors j of a unit (m in base-2 score units).  One work item
-// is (unit b * H_kv + h, query q of the group), items spread round-robin over
-// the CTAs; an item whose unit lies inside one attention CTA's range is
-// skipped (that CTA wrote the output itself); otherwise thread d merges
-// head_dim element d.  The grid is a programmatic dependent of the attention
-// grid: it may become resident early, and griddepcontrol.wait holds it until
-// every attention CTA has finished and its partial stores are visible.
+// over the contributors j of a unit (m in base-2 score units).  CTA c of this
+// grid stands for attention CTA c: for each split unit that CTA holds (at most
+// its first and its last), it merges slice jc of the unit's g x 128 outputs,
+// jc being c's index among the unit's contributors -- so a unit spread over
+// many CTAs is merged by as many.  Each output is one thread's single pass
+// over the contributors (running max, batches of loads in flight), with no
+// CTA barrier.  The grid is a programmatic dependent of the attention
+// grid: its prologue (the length scan) overlaps the attention tail, and
+// griddepcontrol.wait holds it until every attention CTA has finished and its
+// partial stores are visible.
 // ---------------------------------------------------------------------------
-constexpr int kMergeThreads = 128;
-constexpr int kMergeBatch = 8;                        // O loads in flight per thread
+constexpr int kMergeThreads = 256;
+constexpr int kMergeBatch = 8;                        // contributors per batch of loads
 
-__device__ __forceinline__ float merge_block_max(float v, float* red, int warp, int lane) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    const float r = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    __syncthreads();
-    return r;
-}
-__device__ __forceinline__ float merge_block_sum(float v, float* red, int warp, int lane) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    const float r = (red[0] + red[1]) + (red[2] + red[3]);
-    __syncthreads();
-    return r;
-}
-
-__global__ void __launch_bounds__(kMergeThreads, 8) merge_split_units_kernel(const Params p, int n_attn) {
+__global__ void __launch_bounds__(kMergeThreads, 1) merge_split_units_kernel(const Params p, int n_attn) {
     __shared__ int32_t s_lens[kMaxBatchPerLaunch];
     __shared__ int32_t s_prefix[kMaxBatchPerLaunch + 1];
     __shared__ int32_t s_warp_tot[kMergeThreads / 32];
-    __shared__ float s_w[kMergeThreads];
-    __shared__ float s_red[kMergeThreads / 32];
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
@@ -1125,65 +1155,70 @@ __global__ void __launch_bounds__(kMergeThreads, 8) merge_split_units_kernel(con
         if (tid == kMergeThreads - 1) s_prefix[B] = acc;
     }
     __syncthreads();
-    wait_prerequisites();                             // partials are complete and visible from here
     const int64_t T = s_prefix[B];
     const int64_t N = n_attn;
+    const int64_t c = blockIdx.x;
+    const int64_t t_begin = range_start(c, T, N);
+    const int64_t t_end = range_start(c + 1, T, N);
+    if (t_begin >= t_end) return;
     const int g = p.g;
     const int64_t slot_floats = partial_slot_floats(g, 128);
-    const bool dense = T >= N;                        // every CTA range non-empty
-    const int n_items = B * p.Hkv * g;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int ui = item / g;                           // unit b * H_kv + h
-        const int q = item - ui * g;
-        const int b = ui / p.Hkv;
-        Unit u;
-        u.b = b;
-        u.h = ui - b * p.Hkv;
-        u.L = s_lens[b];
-        u.ntb = u.L > 0 ? (u.L + TILE - 1) / TILE : 1;
-        u.U0 = s_prefix[b] + (int64_t)u.h * u.ntb;
-        u.U1 = u.U0 + u.ntb;
-        const int64_t c = cta_of(u.U0, T, N);              // first contributor
-        if (cta_of(u.U1 - 1, T, N) == c) continue;         // inside one CTA's range: not split
+    const bool dense = T >= N;                            // every CTA range non-empty
+    bool waited = false;
+    // the units holding this range's first and last tiles: the only ones it can share
+    for (int which = 0; which < 2; ++which) {
+        const int64_t gt = which == 0 ? t_begin : t_end - 1;
+        const Unit u = find_unit<TILE>(s_prefix, s_lens, B, p.Hkv, gt);
+        if (which == 1 && u.U0 <= t_begin) break;          // the same unit as the first
+        const int64_t c_first = cta_of(u.U0, T, N);
+        if (cta_of(u.U1 - 1, T, N) == c_first) continue;   // inside one range: not split
         const int ncc = unit_contributors(u.U0, u.U1, T, N);
-        const bool first_odd = range_start(c, T, N) < u.U0;   // the unit is c's second unit
-        // dense ranges: contributor j is CTA c + j (slot 2(c + j), or 2c + 1 for
-        // j = 0 when the unit is c's second unit); otherwise the closed form
-        const float* base = p.partials + 2 * c * slot_floats;
+        const bool first_odd = range_start(c_first, T, N) < u.U0;   // the unit is c_first's second unit
+        // this CTA's contributor index, and its slice of the g x 128 outputs
+        const int jc = dense ? (int)(c - c_first) : (int)(t_begin - u.U0);
+        const int per = (g * 128 + ncc - 1) / ncc;
+        const int o0 = jc * per;
+        const int o1 = o0 + per < g * 128 ? o0 + per : g * 128;
+        const float* base = p.partials + 2 * c_first * slot_floats;
         auto part_of = [&](int j) -> const float* {
             if (dense) return base + (2 * (int64_t)j + ((j == 0 && first_odd) ? 1 : 0)) * slot_floats;
-            return p.partials + contributor_slot(j, u.U0, c, first_odd, dense, T, N) * slot_floats;
+            return p.partials + contributor_slot(j, u.U0, c_first, first_odd, dense, T, N) * slot_floats;
         };
-        float mx = -INFINITY;
-        for (int j = tid; j < ncc; j += kMergeThreads) mx = fmaxf(mx, __ldcg(part_of(j) + g * 128 + q));
-        const float M = merge_block_max(mx, s_red, warp, lane);
-        float acc = 0.0f, lsum = 0.0f;
-        for (int j0 = 0; j0 < ncc; j0 += kMergeThreads) {
-            const int j = j0 + tid;
-            float wj = 0.0f;
-            if (j < ncc) {
-                const float* pp = part_of(j);
-                const float m = __ldcg(pp + g * 128 + q);
-                const float l = __ldcg(pp + g * 128 + g + q);
-                wj = (m == -INFINITY) ? 0.0f : fast_exp2(m - M);
-                lsum = fmaf(wj, l, lsum);
-            }
-            s_w[tid] = wj;
-            __syncthreads();
-            const int nj = ncc - j0 < kMergeThreads ? ncc - j0 : kMergeThreads;
-            for (int jj0 = 0; jj0 < nj; jj0 += kMergeBatch) {
-                float v[kMergeBatch];
-#pragma unroll
-                for (int k = 0; k < kMergeBatch; ++k)
-                    v[k] = (jj0 + k < nj) ? __ldcg(part_of(j0 + jj0 + k) + q * 128 + tid) : 0.0f;
-#pragma unroll
-                for (int k = 0; k < kMergeBatch; ++k)
-                    if (jj0 + k < nj) acc = fmaf(s_w[jj0 + k], v[k], acc);
-            }
-            __syncthreads();                               // s_w is reused
+        if (!waited) {
+            wait_prerequisites();                         // partials are complete and visible from here
+            waited = true;
         }
-        const float L = merge_block_sum(lsum, s_red, warp, lane);
-        p.out[((int64_t)u.b * p.Hq + (int64_t)u.h * g + q) * 128 + tid] = L > 0.0f ? acc / L : 0.0f;
+        for (int o = o0 + tid; o < o1; o += kMergeThreads) {
+            const int q = o >> 7, d = o & 127;
+            // one pass over the contributors with a running max (batches of loads in flight)
+            float M = -INFINITY, acc = 0.0f, L = 0.0f;
+            for (int j0 = 0; j0 < ncc; j0 += kMergeBatch) {
+                float m[kMergeBatch], l[kMergeBatch], v[kMergeBatch];
+#pragma unroll
+                for (int k = 0; k < kMergeBatch; ++k) {
+                    const bool in = j0 + k < ncc;
+                    const float* pp = in ? part_of(j0 + k) : base;
+                    m[k] = in ? __ldcg(pp + g * 128 + q) : -INFINITY;
+                    l[k] = in ? __ldcg(pp + g * 128 + g + q) : 0.0f;
+                    v[k] = in ? __ldcg(pp + q * 128 + d) : 0.0f;
+                }
+                float Mb = M;
+#pragma unroll
+                for (int k = 0; k < kMergeBatch; ++k) Mb = fmaxf(Mb, m[k]);
+                if (Mb == -INFINITY) continue;
+                const float f = M == -INFINITY ? 0.0f : fast_exp2(M - Mb);
+                acc *= f;
+                L *= f;
+#pragma unroll
+                for (int k = 0; k < kMergeBatch; ++k) {
+                    const float wk = m[k] == -INFINITY ? 0.0f : fast_exp2(m[k] - Mb);
+                    L = fmaf(wk, l[k], L);
+                    acc = fmaf(wk, v[k], acc);
+                }
+                M = Mb;
+            }
+            p.out[((int64_t)u.b * p.Hq + (int64_t)u.h * g + q) * 128 + d] = L > 0.0f ? acc / L : 0.0f;
+        }
     }
 }
 
