@@ -64,16 +64,15 @@ constexpr int NTERM = 3;                              // E4M3 terms of P
 
 // warp roles, in warpgroups of four (warp w reaches tensor-memory lanes
 // 32 * (w % 4) .. +31, so every group covers the 128 token lanes):
-//   warps  0- 3  K dequant, head_dim  0-63      warps 16-19  V dequant, head_dim 64-127
+//   warps  0- 3, 8-11, 12-15, 16-19  dequant groups 0..3: group i takes the
+//                tiles w = i (mod 4), K and V of one token per thread; it owns
+//                ring stage i and operand buffer i
 //   warps  4- 7  softmax group 0 (queries 0 .. NQ/2-1)
-//   warps  8-11  K dequant, head_dim 64-127     warps 20-23  softmax group 1 (NQ/2 .. NQ-1)
-//   warps 12-15  V dequant, head_dim  0-63      warp 24 loads, 25 Q.K^T MMAs, 26 P.V MMAs,
-//                                               27 the fused append's new tokens
+//   warps 20-23  softmax group 1 (NQ/2 .. NQ-1)
+//   warp 24 loads, 25 Q.K^T MMAs, 26 P.V MMAs, 27 the fused append's new tokens
 constexpr int kS0Warp0 = 4;
-constexpr int kK1Warp0 = 8;
-constexpr int kV0Warp0 = 12;
-constexpr int kV1Warp0 = 16;
 constexpr int kS1Warp0 = 20;
+static_assert(kStages == 4 && kBuf == 4, "one ring stage and one operand buffer per dequant group");
 constexpr int kLoadWarp = 24;
 constexpr int kMmaWarp = 25;                          // Q.K^T
 constexpr int kPvWarp = 26;                           // P.V
@@ -167,6 +166,22 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, int32_
                                           int32_t* status, uint32_t polls) {
     const bool ok = wait_one(bar, parity, abort_flag, status, polls);
     return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// A wait of a 128-thread group: one warp polls the barrier while the other
+// three wait on the group's named barrier without issuing, which then hands
+// every thread the outcome (an AND over the group).
+__device__ __forceinline__ bool group_wait(uint64_t* bar, uint32_t parity, bool poller, int bar_id,
+                                           int32_t* abort_flag, int32_t* status, uint32_t polls) {
+    const bool ok = poller ? wait_warp(bar, parity, abort_flag, status, polls) : true;
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.and.pred po, %2, 128, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)ok), "r"(bar_id)
+        : "memory");
+    return r != 0;
 }
 
 // the softmax warps' named barrier, plain and as an OR-reduction
@@ -564,13 +579,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
     if (warp == kLoadWarp && lane == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.empty[s], 16);
+            mbar_init(&sm.empty[s], 4);
         }
         for (int b = 0; b < kBuf; ++b) {
-            mbar_init(&sm.kfull[b], 8);
+            mbar_init(&sm.kfull[b], 4);
             mbar_init(&sm.qkdone[b], 1);
             mbar_init(&sm.sempty[b], 4 * n_sgrp);
-            mbar_init(&sm.vfull[b], 8);
+            mbar_init(&sm.vfull[b], 4);
             mbar_init(&sm.pfull[b], 4 * n_sgrp);
             mbar_init(&sm.pvdone[b], 1);
         }
@@ -732,118 +747,83 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.appended);
         }
-    } else if (wg == 0 || wg == kK1Warp0 / 4) {
-        // ======== K dequant: head_dim half h of token t's K row ========
-        // Tile w + 1's raw data is read (and its ring stage released) before
-        // tile w's dequant, so that read's latency hides behind the dequant.
+    } else if (!is_softmax) {
+        // ======== dequant group i: tiles w = i (mod 4), K and V of token t ========
+        // A group has four tile periods for each of its tiles, so the latency
+        // of its loads, tensor-memory stores and barriers is spread over four
+        // tiles in flight.  K goes first (its Q.K^T runs ahead of P.V); the
+        // ring stage is released once V's raw data is in registers.
         regs_dec<kRegsDequant>();
-        const int h = wg == 0 ? 0 : 1;                     // head_dim [64h, 64h + 64)
+        const int i = wg == 0 ? 0 : wg - 1;                // wg 0, 2, 3, 4 -> 0, 1, 2, 3
         const int t = 32 * (warp & 3) + lane;              // token, tensor-memory lane
         const uint32_t trow = tbase + ((uint32_t)(32 * (warp & 3)) << 16);
         const uint2* lut_k = &sm.lut[0][0][lane & (kLutCopies - 1)];
-        uint4 xk[2];
-        uint32_t sk = 0;
-        // raw codes and scale bytes of tile w, then its ring stage is released
-        auto fetch = [&](int w) -> bool {
-            const int s = w % kStages;
-            if (!wait_warp(&sm.full[s], ((uint32_t)w / kStages) & 1u, abort_flag, p.status, polls)) return false;
-            const uint8_t* st = sm.ring[s];
+        const uint2* lut_v = &sm.lut[1][0][lane & (kLutCopies - 1)];
+        const uint8_t* st = sm.ring[i];
+        uint8_t* const vdst = sm.vt[i] + (t / 8) * 128 + (t % 8) * 16;
+        const bool poller = (warp & 3) == 0;
+        const int gbar = 3 + i;                            // named barriers 3..6
+        for (int w = i; w < n_work; w += 4) {
+            const uint32_t ph = ((uint32_t)w >> 2) & 1u;
+            if (!group_wait(&sm.full[i], ph, poller, gbar, abort_flag, p.status, polls)) break;
+            // Q.K^T of tile w - 4 has read this K buffer
+            if (w >= 4 && !group_wait(&sm.qkdone[i], ph ^ 1u, poller, gbar, abort_flag, p.status, polls)) break;
+            const uint2 sk = *reinterpret_cast<const uint2*>(st + OFF_KS + t * kSB);
+            uint4 kc[4];
 #pragma unroll
-            for (int j = 0; j < 2; ++j) xk[j] = *reinterpret_cast<const uint4*>(st + t * kKB + 32 * h + 16 * j);
-            sk = *reinterpret_cast<const uint32_t*>(st + OFF_KS + t * kSB + 4 * h);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.empty[s]);
-            return true;
-        };
-        bool ok = n_work > 0 && fetch(0);
-        int w = 0;
-        for (; ok && w < n_work; ++w) {
-            const int b = w % kBuf;
-            const uint32_t ph = ((uint32_t)w / kBuf) & 1u;
-            uint2 l[4];
+            for (int j = 0; j < 4; ++j) kc[j] = *reinterpret_cast<const uint4*>(st + t * kKB + 16 * j);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) l[i] = lut_k[((sk >> (8 * i)) & 0x7F) * kLutCopies];
-            const uint4 c0 = xk[0], c1 = xk[1];
-            if (w + 1 < n_work) ok = fetch(w + 1);
-            // Q.K^T of tile w - kBuf has read this K buffer
-            if (!ok || (w >= kBuf && !wait_warp(&sm.qkdone[b], ph ^ 1u, abort_flag, p.status, polls))) {
-                ok = false;
-                break;
+            for (int hh = 0; hh < 2; ++hh) {               // head_dim 64hh .. 64hh + 63
+                const uint32_t sc = hh ? sk.y : sk.x;
+                uint2 l[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) l[k] = lut_k[((sc >> (8 * k)) & 0x7F) * kLutCopies];
+                const uint4 c0 = kc[2 * hh], c1 = kc[2 * hh + 1];
+                uint32_t kf[16];                           // 64 codes -> 16 columns (4 FP8 each)
+                dequant_word(c0.x, l[0].x, l[0].y, kf[0], kf[1]);
+                dequant_word(c0.y, l[0].x, l[0].y, kf[2], kf[3]);
+                dequant_word(c0.z, l[1].x, l[1].y, kf[4], kf[5]);
+                dequant_word(c0.w, l[1].x, l[1].y, kf[6], kf[7]);
+                dequant_word(c1.x, l[2].x, l[2].y, kf[8], kf[9]);
+                dequant_word(c1.y, l[2].x, l[2].y, kf[10], kf[11]);
+                dequant_word(c1.z, l[3].x, l[3].y, kf[12], kf[13]);
+                dequant_word(c1.w, l[3].x, l[3].y, kf[14], kf[15]);
+                tmem_st_x16(trow + C::COL_K + 32 * i + 16 * hh, kf);
             }
-            // 64 codes -> 16 tensor-memory columns (4 FP8 each)
-            uint32_t kf[16];
-            dequant_word(c0.x, l[0].x, l[0].y, kf[0], kf[1]);
-            dequant_word(c0.y, l[0].x, l[0].y, kf[2], kf[3]);
-            dequant_word(c0.z, l[1].x, l[1].y, kf[4], kf[5]);
-            dequant_word(c0.w, l[1].x, l[1].y, kf[6], kf[7]);
-            dequant_word(c1.x, l[2].x, l[2].y, kf[8], kf[9]);
-            dequant_word(c1.y, l[2].x, l[2].y, kf[10], kf[11]);
-            dequant_word(c1.z, l[3].x, l[3].y, kf[12], kf[13]);
-            dequant_word(c1.w, l[3].x, l[3].y, kf[14], kf[15]);
-            tmem_st_x16(trow + C::COL_K + 32 * b + 16 * h, kf);
+            const uint2 sv = *reinterpret_cast<const uint2*>(st + OFF_VS + t * kSB);
+            uint4 vc[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) vc[j] = *reinterpret_cast<const uint4*>(st + OFF_VC + t * kKB + 16 * j);
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.kfull[b]);     // Q.K^T of tile w may start
-        }
-    } else if (wg == kV0Warp0 / 4 || wg == kV1Warp0 / 4) {
-        // ======== V dequant: head_dim half h of token t's V row -> V^T ========
-        // Reads tile w + 1's raw data ahead, like the K warps.
-        regs_dec<kRegsDequant>();
-        const int h = wg == kV0Warp0 / 4 ? 0 : 1;
-        const int t = 32 * (warp & 3) + lane;              // token
-        const int rot = (t >> 1) & 1;                      // chunk order: fewer bank conflicts
-        const uint2* lut_v = &sm.lut[1][0][lane & (kLutCopies - 1)];
-        uint4 xv[2];
-        uint32_t sv = 0;
-        auto fetch = [&](int w) -> bool {
-            const int s = w % kStages;
-            if (!wait_warp(&sm.full[s], ((uint32_t)w / kStages) & 1u, abort_flag, p.status, polls)) return false;
-            const uint8_t* st = sm.ring[s];
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-                xv[j] = *reinterpret_cast<const uint4*>(st + OFF_VC + t * kKB + 32 * h + 16 * (j ^ rot));
-            sv = *reinterpret_cast<const uint32_t*>(st + OFF_VS + t * kSB + 4 * h);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.empty[s]);
-            return true;
-        };
-        bool ok = n_work > 0 && fetch(0);
-        int w = 0;
-        for (; ok && w < n_work; ++w) {
-            const int b = w % kBuf;
-            const uint32_t ph = ((uint32_t)w / kBuf) & 1u;
-            // lookup words of chunk j (head_dim 64h + 32(j ^ rot) ..): its two blocks
-            uint2 l[4];
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int cc = j ^ rot;
-                l[2 * j] = lut_v[((sv >> (16 * cc)) & 0x7F) * kLutCopies];
-                l[2 * j + 1] = lut_v[((sv >> (16 * cc + 8)) & 0x7F) * kLutCopies];
+            if (lane == 0) {
+                mbar_arrive(&sm.kfull[i]);                 // Q.K^T of tile w may start
+                mbar_arrive(&sm.empty[i]);                 // the loader may refill stage i
             }
-            const uint4 c[2] = {xv[0], xv[1]};
-            if (w + 1 < n_work) ok = fetch(w + 1);
-            // P.V of tile w - kBuf has read this V^T buffer
-            if (!ok || (w >= kBuf && !wait_warp(&sm.pvdone[b], ph ^ 1u, abort_flag, p.status, polls))) {
-                ok = false;
-                break;
-            }
-            // 64 codes -> 4 rows of 16 head_dim bytes of V^T
-            uint8_t* dst = sm.vt[b] + (4 * h) * 2048 + (t / 8) * 128 + (t % 8) * 16;
+            // P.V of tile w - 4 has read this V^T buffer
+            if (w >= 4 && !group_wait(&sm.pvdone[i], ph ^ 1u, poller, gbar, abort_flag, p.status, polls)) break;
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int cc = j ^ rot;
-                uint4 o0, o1;
-                dequant_word(c[j].x, l[2 * j].x, l[2 * j].y, o0.x, o0.y);
-                dequant_word(c[j].y, l[2 * j].x, l[2 * j].y, o0.z, o0.w);
-                dequant_word(c[j].z, l[2 * j + 1].x, l[2 * j + 1].y, o1.x, o1.y);
-                dequant_word(c[j].w, l[2 * j + 1].x, l[2 * j + 1].y, o1.z, o1.w);
-                *reinterpret_cast<uint4*>(dst + (2 * cc) * 2048) = o0;
-                *reinterpret_cast<uint4*>(dst + (2 * cc + 1) * 2048) = o1;
+            for (int hh = 0; hh < 2; ++hh) {
+                const uint32_t sc = hh ? sv.y : sv.x;
+                uint2 l[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) l[k] = lut_v[((sc >> (8 * k)) & 0x7F) * kLutCopies];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {              // 32 codes -> 2 rows of 16 head_dim bytes of V^T
+                    const uint4 c = vc[2 * hh + j];
+                    uint4 o0, o1;
+                    dequant_word(c.x, l[2 * j].x, l[2 * j].y, o0.x, o0.y);
+                    dequant_word(c.y, l[2 * j].x, l[2 * j].y, o0.z, o0.w);
+                    dequant_word(c.z, l[2 * j + 1].x, l[2 * j + 1].y, o1.x, o1.y);
+                    dequant_word(c.w, l[2 * j + 1].x, l[2 * j + 1].y, o1.z, o1.w);
+                    *reinterpret_cast<uint4*>(vdst + (4 * hh + 2 * j) * 2048) = o0;
+                    *reinterpret_cast<uint4*>(vdst + (4 * hh + 2 * j + 1) * 2048) = o1;
+                }
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.vfull[b]);     // P.V of tile w may start
+            if (lane == 0) mbar_arrive(&sm.vfull[i]);     // P.V of tile w may start
         }
     } else if (is_softmax && sgrp >= n_sgrp) {
         // a group with padding queries only: nothing to do (its P columns stay
@@ -910,40 +890,61 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
                 l_run[q] = 0.0f;
             }
             bool any_pv = false;
-            for (int64_t gt = seg_lo; gt < seg_hi; ++gt) {
-                const int valid = tile_valid(u, gt);
-                if (valid <= 0) continue;
-                const int b = (int)(w % kBuf);
-                const uint32_t ph = (w / kBuf) & 1u;
-                float s[NH];
-                if (!aborted && !wait_warp(&sm.qkdone[b], ph, abort_flag, p.status, polls)) aborted = true;
+            // Two tiles per pass where the segment has them: every wait, barrier
+            // and fence of the pass is shared by both, so its latency is paid
+            // once per 256 tokens.
+            for (int64_t gt = seg_lo; gt < seg_hi;) {
+                const int valid0 = tile_valid(u, gt);
+                if (valid0 <= 0) {                         // the empty tile of a zero-length sequence
+                    ++gt;
+                    continue;
+                }
+                // every other tile of a unit is full or its last, so the second
+                // tile (when the segment has one) has work too
+                const bool two = gt + 1 < seg_hi;
+                const int valid1 = two ? tile_valid(u, gt + 1) : 0;
+                const int b0 = (int)(w % kBuf), b1 = (int)((w + 1) % kBuf);
+                const uint32_t ph0 = (w / kBuf) & 1u, ph1 = ((w + 1) / kBuf) & 1u;
+                float s0[NH], s1[NH];
+                if (!aborted && !wait_warp(&sm.qkdone[b0], ph0, abort_flag, p.status, polls)) aborted = true;
+                if (!aborted && two && !wait_warp(&sm.qkdone[b1], ph1, abort_flag, p.status, polls)) aborted = true;
                 if (!aborted) {
                     tc::fence_after_sync();
-                    uint32_t rh[NH], rl[NH];
-                    tmem_ld_cols<NH>(trow + C::COL_S + NS * b + q0, rh);
-                    tmem_ld_cols<NH>(trow + C::COL_S + NS * b + NQ + q0, rl);
+                    uint32_t rh0[NH], rl0[NH], rh1[NH], rl1[NH];
+                    tmem_ld_cols<NH>(trow + C::COL_S + NS * b0 + q0, rh0);
+                    tmem_ld_cols<NH>(trow + C::COL_S + NS * b0 + NQ + q0, rl0);
+                    if (two) {
+                        tmem_ld_cols<NH>(trow + C::COL_S + NS * b1 + q0, rh1);
+                        tmem_ld_cols<NH>(trow + C::COL_S + NS * b1 + NQ + q0, rl1);
+                    }
                     tc::tmem_wait_ld();
                     tc::fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.sempty[b]);
-                    const bool live = t < valid;
+                    if (lane == 0) {
+                        mbar_arrive(&sm.sempty[b0]);
+                        if (two) mbar_arrive(&sm.sempty[b1]);
+                    }
+                    const bool live0 = t < valid0, live1 = t < valid1;
 #pragma unroll
-                    for (int q = 0; q < NH; ++q)
-                        s[q] = live ? fmaf(__uint_as_float(rl[q]), 0.0625f, __uint_as_float(rh[q])) * cs[q]
-                                    : -INFINITY;
+                    for (int q = 0; q < NH; ++q) {
+                        s0[q] = live0 ? fmaf(__uint_as_float(rl0[q]), 0.0625f, __uint_as_float(rh0[q])) * cs[q]
+                                      : -INFINITY;
+                        s1[q] = live1 ? fmaf(__uint_as_float(rl1[q]), 0.0625f, __uint_as_float(rh1[q])) * cs[q]
+                                      : -INFINITY;
+                    }
                 } else {
 #pragma unroll
-                    for (int q = 0; q < NH; ++q) s[q] = -INFINITY;
+                    for (int q = 0; q < NH; ++q) s0[q] = s1[q] = -INFINITY;
                 }
                 bool need = false;
 #pragma unroll
-                for (int q = 0; q < NH; ++q) need |= s[q] > m_run[q] + kRescaleSlack;
+                for (int q = 0; q < NH; ++q) need |= fmaxf(s0[q], s1[q]) > m_run[q] + kRescaleSlack;
                 if (softmax_any(need, bar_id)) {
-                    // raise the running max to the tile max (per query over the 128
-                    // tokens), rescale l and this group's O columns
+                    // raise the running max to the max over the pass's tokens (per
+                    // query), rescale l and this group's O columns
 #pragma unroll
                     for (int q = 0; q < NH; ++q) {
-                        float mx = s[q];
+                        float mx = fmaxf(s0[q], s1[q]);
 #pragma unroll
                         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
                         if (lane == 0) sm.red[sw][q0 + q] = mx;
@@ -980,45 +981,65 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
                         }
                     }
                 }
-                // P terms of this token for this group's queries: column n = k * NQ + q0 + q
-                uint32_t tw[NTERM][NH / 4];
+                // P terms of this thread's token in both tiles for this group's
+                // queries: column n = k * NQ + q0 + q
+                uint32_t tw0[NTERM][NH / 4], tw1[NTERM][NH / 4];
 #pragma unroll
                 for (int q = 0; q < NH; q += 4) {
-                    uint32_t ta[NTERM], tb[NTERM];
-                    float pq[4];
+                    uint32_t ta[NTERM], tb[NTERM], tc_[NTERM], td[NTERM];
+                    float pa[4], pb_[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        pq[i] = (m_run[q + i] == -INFINITY) ? 0.0f : fast_exp2(s[q + i] - m_run[q + i]);
-                        l_run[q + i] += pq[i];
+                        const bool none = m_run[q + i] == -INFINITY;
+                        pa[i] = none ? 0.0f : fast_exp2(s0[q + i] - m_run[q + i]);
+                        pb_[i] = none ? 0.0f : fast_exp2(s1[q + i] - m_run[q + i]);
+                        l_run[q + i] += pa[i] + pb_[i];
                     }
-                    p_terms(pq[0], pq[1], ta);
-                    p_terms(pq[2], pq[3], tb);
+                    p_terms(pa[0], pa[1], ta);
+                    p_terms(pa[2], pa[3], tb);
+                    p_terms(pb_[0], pb_[1], tc_);
+                    p_terms(pb_[2], pb_[3], td);
 #pragma unroll
-                    for (int k = 0; k < NTERM; ++k) tw[k][q / 4] = ta[k] | (tb[k] << 16);
+                    for (int k = 0; k < NTERM; ++k) {
+                        tw0[k][q / 4] = ta[k] | (tb[k] << 16);
+                        tw1[k][q / 4] = tc_[k] | (td[k] << 16);
+                    }
                 }
-                // P.V of tile w - kBuf has read this P buffer
+                // P.V of tiles w - kBuf and w + 1 - kBuf have read these P buffers
                 if (!aborted && w >= (uint32_t)kBuf &&
-                    !wait_warp(&sm.pvdone[b], ph ^ 1u, abort_flag, p.status, polls))
+                    !wait_warp(&sm.pvdone[b0], ph0 ^ 1u, abort_flag, p.status, polls))
+                    aborted = true;
+                if (!aborted && two && w + 1 >= (uint32_t)kBuf &&
+                    !wait_warp(&sm.pvdone[b1], ph1 ^ 1u, abort_flag, p.status, polls))
                     aborted = true;
                 if (!aborted) {
-                    uint8_t* dst = sm.pb[b] + (t / 8) * 128 + (t % 8) * 16;
+                    uint8_t* dst0 = sm.pb[b0] + (t / 8) * 128 + (t % 8) * 16;
+                    uint8_t* dst1 = sm.pb[b1] + (t / 8) * 128 + (t % 8) * 16;
 #pragma unroll
                     for (int k = 0; k < NTERM; ++k) {
                         const int n = k * NQ + q0;
                         if constexpr (NH == 4) {
-                            *reinterpret_cast<uint32_t*>(dst + (n / 16) * 2048 + (n % 16)) = tw[k][0];
+                            *reinterpret_cast<uint32_t*>(dst0 + (n / 16) * 2048 + (n % 16)) = tw0[k][0];
+                            if (two) *reinterpret_cast<uint32_t*>(dst1 + (n / 16) * 2048 + (n % 16)) = tw1[k][0];
                         } else {
-                            *reinterpret_cast<uint2*>(dst + (n / 16) * 2048 + (n % 16)) =
-                                make_uint2(tw[k][0], tw[k][1]);
+                            *reinterpret_cast<uint2*>(dst0 + (n / 16) * 2048 + (n % 16)) =
+                                make_uint2(tw0[k][0], tw0[k][1]);
+                            if (two)
+                                *reinterpret_cast<uint2*>(dst1 + (n / 16) * 2048 + (n % 16)) =
+                                    make_uint2(tw1[k][0], tw1[k][1]);
                         }
                     }
                     fence_proxy_async_smem();
                     tc::fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.pfull[b]);
+                    if (lane == 0) {
+                        mbar_arrive(&sm.pfull[b0]);
+                        if (two) mbar_arrive(&sm.pfull[b1]);
+                    }
                 }
                 any_pv = true;
-                ++w;
+                w += two ? 2u : 1u;
+                gt += two ? 2 : 1;
             }
 
             // ---- segment end ----
