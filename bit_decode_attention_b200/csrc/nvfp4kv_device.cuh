@@ -71,11 +71,65 @@ __device__ __forceinline__ float e2m1_magnitude(uint32_t m3) {
 // +-6; the sign bit is copied (negative values rounding to 0 give 0x8).  The
 // comparisons are against the exact midpoints of the grid, strict where the
 // lower neighbour has the even code and inclusive where the upper one has.
+// NaN gives 0x7.
 __device__ __forceinline__ uint32_t e2m1_from_float(float y) {
+    if (y != y) return 0x7u;
     const float a = fabsf(y);
     uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) +
                  (a > 2.5f) + (a >= 3.5f) + (a > 5.0f);
     return c | ((__float_as_uint(y) >> 28) & 0x8u);
+}
+
+// Two finite floats -> two E2M1 codes in one byte (lo in the low nibble), by
+// the hardware conversion: round to nearest even, saturating at +-6, the sign
+// kept on zero -- the rule of e2m1_from_float for every finite input.
+__device__ __forceinline__ uint32_t e2m1x2_from_floats(float lo, float hi) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r)
+        : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Two lanes of fp32 in one 64-bit register, for the paired IEEE arithmetic
+// of sm_100 (each lane rounded to nearest even on its own, no flush to zero).
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t x, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+}
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// a / b rounded to nearest even, from y = RN(1/b), for normal b and normal
+// y with no overflow: Markstein's division by correction (P. Markstein, "IA-64
+// and Elementary Functions", 2000).  One correction of q0 = RN(a y) leaves a
+// quotient within one ulp of a/b, whose residual a - b q is then exact in a
+// fused multiply-add; with y the correctly rounded reciprocal, the second
+// correction RN(q + (a - b q) y) is the correctly rounded quotient.
+__device__ __forceinline__ float div_rn_by_correction(float a, float b, float y) {
+    const float q0 = __fmul_rn(a, y);
+    const float q1 = __fmaf_rn(__fmaf_rn(-q0, b, a), y, q0);
+    return __fmaf_rn(__fmaf_rn(-q1, b, a), y, q1);
+}
+// The same for two dividends at once (yy = (y, y), nb = (-b, -b)); the
+// quotients come back with the signs of their dividends, zeros included.
+__device__ __forceinline__ uint64_t div2_rn_by_correction(uint64_t a, uint64_t nb, uint64_t yy) {
+    const uint64_t q0 = f32x2_mul(a, yy);
+    const uint64_t q1 = f32x2_fma(f32x2_fma(q0, nb, a), yy, q0);
+    const uint64_t q2 = f32x2_fma(f32x2_fma(q1, nb, a), yy, q1);
+    return q2 | (a & 0x8000000080000000ull);
 }
 
 // ---------------------------------------------------------------------------
@@ -110,27 +164,51 @@ __device__ __forceinline__ void load16(const void* x, int64_t elem, float (&v)[1
 }
 
 // Quantize one micro-block: returns the scale byte, writes 8 packed bytes.
+// The codes are E2M1(RN(v / den)) element by element.  A block with a NaN or
+// an infinity, a saturated scale (amax / (6 s_tensor) > 448), or a den that is
+// zero, subnormal or near the ends of the fp32 range takes the IEEE division
+// and the comparison encoder; every other block divides by correction from
+// one reciprocal and encodes two elements per hardware conversion -- the same
+// codes, bit for bit.
 __device__ __forceinline__ uint32_t quantize_block(const float (&v)[16], float s_tensor, uint2& packed) {
     float amax = 0.0f;
+    bool nan = false;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    for (int i = 0; i < 16; ++i) {
+        amax = fmaxf(amax, fabsf(v[i]));
+        nan |= v[i] != v[i];
+    }
     const float d6 = __fmul_rn(6.0f, s_tensor);
     const float r = __fdiv_rn(amax, d6);
     const uint32_t sb = e4m3_from_float(r);
     const float den = __fmul_rn(e4m3_to_float(sb), s_tensor);
-    uint32_t c[16];
-    if (den == 0.0f) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) c[i] = (__float_as_uint(v[i]) >> 28) & 0x8u;
-    } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) c[i] = e2m1_from_float(__fdiv_rn(v[i], den));
-    }
     uint32_t lo = 0, hi = 0;
+    // r <= 448 bounds every |v / den| near 6, far from overflow
+    if (!nan && r <= 448.0f && den >= 0x1p-125f && den <= 0x1p125f) {
+        const float y = __frcp_rn(den);
+        uint32_t byte[8];
+        // copysignf: a zero quotient keeps the sign of its dividend (the
+        // corrections add +0 to -0)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        lo |= c[i] << (4 * i);
-        hi |= c[8 + i] << (4 * i);
+        for (int k = 0; k < 8; ++k)
+            byte[k] = e2m1x2_from_floats(copysignf(div_rn_by_correction(v[2 * k], den, y), v[2 * k]),
+                                         copysignf(div_rn_by_correction(v[2 * k + 1], den, y), v[2 * k + 1]));
+        lo = __byte_perm(byte[0] | (byte[1] << 8), byte[2] | (byte[3] << 8), 0x5410);
+        hi = __byte_perm(byte[4] | (byte[5] << 8), byte[6] | (byte[7] << 8), 0x5410);
+    } else {
+        uint32_t c[16];
+        if (den == 0.0f) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) c[i] = (__float_as_uint(v[i]) >> 28) & 0x8u;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) c[i] = e2m1_from_float(__fdiv_rn(v[i], den));
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            lo |= c[i] << (4 * i);
+            hi |= c[8 + i] << (4 * i);
+        }
     }
     packed = make_uint2(lo, hi);
     return sb;

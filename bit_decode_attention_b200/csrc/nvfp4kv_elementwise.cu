@@ -90,124 +90,255 @@ cudaError_t launch_calib(const void* x, bool f32, int64_t n, float* d_s_tensor, 
 }
 
 // ---------------------------------------------------------------------------
-// Quantize + append.  One thread per 16-element micro-block; threads are
-// ordered (b, h, t, block) so that code and scale writes are contiguous in
-// the [B][H_kv][S_max][...] planes.
+// Index arithmetic.  Division by a launch-invariant divisor (T. Granlund and
+// P. Montgomery, "Division by Invariant Integers using Multiplication", 1994):
+// for 1 <= d < 2^31 and 0 <= x < 2^31, x / d = (umulhi(x, m) + x) >> l with
+// l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1 (mod 2^32).  A
+// runtime 32-bit division is a software routine of a few dozen instructions;
+// this is two.
 // ---------------------------------------------------------------------------
-// Quantize-append of one plane (a1-a4); `item` enumerates (b, t, h, blk)
-// with blk fastest.  Index math in 32 bits when the item count fits.
+struct FastDiv {
+    uint32_t d, m, l;
+    FastDiv() = default;
+    __host__ explicit FastDiv(uint32_t d_) : d(d_), m(0), l(0) {
+        while ((1ull << l) < d) ++l;
+        m = (uint32_t)((((1ull << 32) * ((1ull << l) - d)) / d + 1) & 0xFFFFFFFFull);
+    }
+    __device__ __forceinline__ uint32_t div(uint32_t x) const { return (__umulhi(x, m) + x) >> l; }
+};
+
+// launch-invariant shape of a quantize (nblk = elements per row / block size,
+// a power of two)
+struct QShape {
+    int B, n_new, Hkv, D, S_max, lg_nblk;
+    FastDiv fd_hkv, fd_new;
+};
+
+__host__ inline QShape make_qshape(int B, int n_new, int Hkv, int D, int S_max, int block) {
+    QShape q;
+    q.B = B; q.n_new = n_new; q.Hkv = Hkv; q.D = D; q.S_max = S_max;
+    q.lg_nblk = 0;
+    while ((block << q.lg_nblk) < D) ++q.lg_nblk;
+    q.fd_hkv = FastDiv((uint32_t)Hkv);
+    q.fd_new = FastDiv((uint32_t)n_new);
+    return q;
+}
+
+// item i enumerates (b, t, h, blk), blk fastest: the order of the input
+// [B][n_new][H_kv][D], so item i starts at element i * block
+struct QItem {
+    int b, t, h, blk;
+};
+__device__ __forceinline__ QItem decode_item(const QShape& q, uint32_t i) {
+    QItem it;
+    it.blk = (int)(i & ((1u << q.lg_nblk) - 1u));
+    const uint32_t r = i >> q.lg_nblk;                 // (b * n_new + t) * Hkv + h
+    const uint32_t bt = q.fd_hkv.div(r);
+    it.h = (int)(r - bt * (uint32_t)q.Hkv);
+    it.b = (int)q.fd_new.div(bt);
+    it.t = (int)(bt - (uint32_t)it.b * (uint32_t)q.n_new);
+    return it;
+}
+__device__ __forceinline__ QItem decode_item(const QShape& q, int64_t i) {
+    QItem it;
+    it.blk = (int)(i & ((1 << q.lg_nblk) - 1));
+    int64_t r = i >> q.lg_nblk;
+    it.h = (int)(r % q.Hkv);
+    r /= q.Hkv;
+    it.t = (int)(r % q.n_new);
+    it.b = (int)(r / q.n_new);
+    return it;
+}
+
+// ---------------------------------------------------------------------------
+// Per-CTA constants of a tensor scale s: for every scale byte sb, the block
+// divisor den = RN(value(sb) * s), its reciprocal RN(1/den) and whether den
+// is in the range where quantize_block's division by correction applies; and
+// the reciprocal of d6 = RN(6 s) with the same range test.
+// ---------------------------------------------------------------------------
+struct QTable {
+    float den[128], rcp[128];
+    uint32_t fast[4];                                  // bit sb: den in range
+    float d6, rcp_d6;
+    bool d6_fast;
+};
+
+__device__ __forceinline__ bool correction_range(float d) { return d >= 0x1p-125f && d <= 0x1p125f; }
+
+// all threads of the CTA; a barrier follows
+__device__ __forceinline__ void build_qtable(QTable& tb, float st) {
+    for (int sb = threadIdx.x; sb < 128; sb += blockDim.x) {
+        const float den = __fmul_rn(e4m3_to_float((uint32_t)sb), st);
+        tb.den[sb] = den;
+        tb.rcp[sb] = correction_range(den) ? __frcp_rn(den) : 0.0f;
+        const uint32_t bit = __ballot_sync(__activemask(), correction_range(den));
+        if ((threadIdx.x & 31) == 0 && sb < 128) tb.fast[sb >> 5] = bit;
+    }
+    if (threadIdx.x == 0) {
+        tb.d6 = __fmul_rn(6.0f, st);
+        tb.d6_fast = correction_range(tb.d6);
+        tb.rcp_d6 = tb.d6_fast ? __frcp_rn(tb.d6) : 0.0f;
+    }
+}
+
+// quantize_block with the tensor-scale constants from the table: the same
+// codes and scale byte, bit for bit (the per-block IEEE divisions are
+// replaced by divisions by correction where those are exact)
+__device__ __forceinline__ uint32_t quantize_block_tab(const float (&v)[16], const QTable& tb, float st,
+                                                       uint2& packed) {
+    // the block maximum, NaN if an element is NaN (max.NaN propagates it)
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) asm("max.NaN.f32 %0, %0, %1;" : "+f"(amax) : "f"(fabsf(v[i])));
+    // r = RN(amax / d6): by correction when d6 is in range and amax finite; a
+    // quotient past 448 (or an overflow, or a NaN) goes to the general path
+    const float r = (tb.d6_fast && amax <= 3.4028234663852886e38f)
+                        ? div_rn_by_correction(amax, tb.d6, tb.rcp_d6)
+                        : 1e30f;
+    if (r <= 448.0f) {
+        const uint32_t sb = e4m3_from_float(r);
+        if ((tb.fast[sb >> 5] >> (sb & 31)) & 1u) {
+            const float den = tb.den[sb], y = tb.rcp[sb];
+            const uint64_t nb = f32x2_pack(-den, -den), yy = f32x2_pack(y, y);
+            uint32_t byte[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                float q0, q1;
+                f32x2_unpack(div2_rn_by_correction(f32x2_pack(v[2 * k], v[2 * k + 1]), nb, yy), q0, q1);
+                byte[k] = e2m1x2_from_floats(q0, q1);
+            }
+            packed = make_uint2(__byte_perm(byte[0] | (byte[1] << 8), byte[2] | (byte[3] << 8), 0x5410),
+                                __byte_perm(byte[4] | (byte[5] << 8), byte[6] | (byte[7] << 8), 0x5410));
+            return sb;
+        }
+    }
+    return quantize_block(v, st, packed);
+}
+
+// ---------------------------------------------------------------------------
+// Quantize + append.  One thread per 16-element micro-block; consecutive
+// threads take consecutive blocks of the input, and the code and scale writes
+// of a token row are contiguous in the [B][H_kv][S_max][...] planes.
+// ---------------------------------------------------------------------------
+// Quantize-append of one block (a1-a4).
 template <bool F32, typename I>
 __device__ __forceinline__ void quantize_append_item(
-    const void* __restrict__ x_new, I i, int B, int n_new, int Hkv, int D,
-    const int32_t* __restrict__ start_pos, int32_t* __restrict__ new_lens, float st, bool st_ok,
-    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int S_max, int32_t* __restrict__ status) {
-    const int nblk = D / 16;
-    const int blk = (int)(i % nblk);
-    I r = i / nblk;
-    const int t = (int)(r % n_new);
-    r /= n_new;
-    const int h = (int)(r % Hkv);
-    const int b = (int)(r / Hkv);
-    const bool leader = (t == 0 && h == 0 && blk == 0);
+    const void* __restrict__ x_new, I i, const QShape& q, const int32_t* __restrict__ start_pos,
+    int32_t* __restrict__ new_lens, float st, bool st_ok, const QTable& tb, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales, int32_t* __restrict__ status) {
+    const QItem it = decode_item(q, i);
+    const bool leader = (it.t == 0 && it.h == 0 && it.blk == 0);
     if (!st_ok) {
         if (i == 0) report(status, NVFP4_ERR_NONFINITE);
         return;
     }
-    const int start = start_pos[b];
-    if (start < 0 || (int64_t)start + n_new > S_max) {
+    const int start = start_pos[it.b];
+    if (start < 0 || (int64_t)start + q.n_new > q.S_max) {
         if (leader) report(status, NVFP4_ERR_CAPACITY);
         return;
     }
-    if (leader && new_lens != nullptr) new_lens[b] = start + n_new;
+    if (leader && new_lens != nullptr) new_lens[it.b] = start + q.n_new;
     float v[16];
-    load16<F32>(x_new, (((int64_t)b * n_new + t) * Hkv + h) * D + 16 * blk, v);
+    load16<F32>(x_new, (int64_t)i * 16, v);
     uint2 packed;
-    const uint32_t sb = quantize_block(v, st, packed);
-    const int64_t slot = ((int64_t)b * Hkv + h) * S_max + start + t;
-    *reinterpret_cast<uint2*>(codes + slot * (D / 2) + 8 * blk) = packed;
-    scales[slot * (D / 16) + blk] = (uint8_t)sb;
+    const uint32_t sb = quantize_block_tab(v, tb, st, packed);
+    const int64_t slot = ((int64_t)it.b * q.Hkv + it.h) * q.S_max + start + it.t;
+    *reinterpret_cast<uint2*>(codes + slot * (q.D / 2) + 8 * it.blk) = packed;
+    scales[slot * (q.D / 16) + it.blk] = (uint8_t)sb;
 }
 
 // One launch for the K and V planes of the same tokens: blockIdx.y selects the
 // plane (0: K, which also writes new_lens; 1: V).
 template <bool F32>
 __global__ void __launch_bounds__(256) quantize_append_kv_kernel(
-    const void* __restrict__ x_k, const void* __restrict__ x_v, int B, int n_new, int Hkv, int D,
+    const void* __restrict__ x_k, const void* __restrict__ x_v, const QShape q,
     const int32_t* __restrict__ start_pos, int32_t* __restrict__ new_lens,
     const float* __restrict__ st_k_p, const float* __restrict__ st_v_p,
     uint8_t* __restrict__ codes_k, uint8_t* __restrict__ scales_k, uint8_t* __restrict__ codes_v,
-    uint8_t* __restrict__ scales_v, int S_max, int32_t* __restrict__ status) {
+    uint8_t* __restrict__ scales_v, int32_t* __restrict__ status) {
+    __shared__ QTable tb;
     const bool is_v = blockIdx.y == 1;
     const float st = *(is_v ? st_v_p : st_k_p);
     const bool st_ok = st > 0.0f && st <= 3.4028234663852886e38f;  // finite and positive
-    const int64_t total = (int64_t)B * Hkv * n_new * (D / 16);
+    build_qtable(tb, st);
+    __syncthreads();
+    const int64_t total = ((int64_t)q.B * q.Hkv * q.n_new) << q.lg_nblk;
     const void* x = is_v ? x_v : x_k;
     uint8_t* codes = is_v ? codes_v : codes_k;
     uint8_t* scales = is_v ? scales_v : scales_k;
     int32_t* nl = is_v ? nullptr : new_lens;
     if (total < (int64_t)INT32_MAX) {
-        for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < (int)total; i += gridDim.x * blockDim.x)
-            quantize_append_item<F32, int>(x, i, B, n_new, Hkv, D, start_pos, nl, st, st_ok, codes, scales,
-                                           S_max, status);
+        for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < (uint32_t)total; i += gridDim.x * blockDim.x)
+            quantize_append_item<F32, uint32_t>(x, i, q, start_pos, nl, st, st_ok, tb, codes, scales, status);
     } else {
         for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
              i += (int64_t)gridDim.x * blockDim.x)
-            quantize_append_item<F32, int64_t>(x, i, B, n_new, Hkv, D, start_pos, nl, st, st_ok, codes,
-                                               scales, S_max, status);
+            quantize_append_item<F32, int64_t>(x, i, q, start_pos, nl, st, st_ok, tb, codes, scales, status);
     }
 }
 
 // With a block table (paged planes), token slot `pos` of sequence b is slot
 // pos % page_tokens of pool page block_table[b * max_pages + pos / page_tokens]
 // (pool layout [page][Hkv][page_tokens][...]) and S_max = max_pages * page_tokens.
+template <bool F32, typename I>
+__device__ __forceinline__ void quantize_append_paged_item(
+    const void* __restrict__ x_new, I i, const QShape& q, const int32_t* __restrict__ start_pos,
+    int32_t* __restrict__ new_lens, float st, bool st_ok, const QTable& tb, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales, int32_t* __restrict__ status, const int32_t* __restrict__ block_table,
+    int page_tokens, int max_pages, int num_pages) {
+    const QItem it = decode_item(q, i);
+    const bool leader = (it.t == 0 && it.h == 0 && it.blk == 0);
+    if (!st_ok) {
+        if (i == 0) report(status, NVFP4_ERR_NONFINITE);
+        return;
+    }
+    const int start = start_pos[it.b];
+    if (start < 0 || (int64_t)start + q.n_new > q.S_max) {
+        if (leader) report(status, NVFP4_ERR_CAPACITY);
+        return;
+    }
+    if (leader && new_lens != nullptr) new_lens[it.b] = start + q.n_new;
+    int64_t slot;
+    if (block_table == nullptr) {
+        slot = ((int64_t)it.b * q.Hkv + it.h) * q.S_max + start + it.t;
+    } else {
+        const int pos = start + it.t;
+        const int page = block_table[(int64_t)it.b * max_pages + pos / page_tokens];
+        if (page < 0 || page >= num_pages) {
+            report(status, NVFP4_ERR_INVALID_ARG);
+            return;
+        }
+        slot = ((int64_t)page * q.Hkv + it.h) * page_tokens + pos % page_tokens;
+    }
+    float v[16];
+    load16<F32>(x_new, (int64_t)i * 16, v);
+    uint2 packed;
+    const uint32_t sb = quantize_block_tab(v, tb, st, packed);
+    *reinterpret_cast<uint2*>(codes + slot * (q.D / 2) + 8 * it.blk) = packed;
+    scales[slot * (q.D / 16) + it.blk] = (uint8_t)sb;
+}
+
 template <bool F32>
 __global__ void __launch_bounds__(256) quantize_append_kernel(
-    const void* __restrict__ x_new, int B, int n_new, int Hkv, int D,
-    const int32_t* __restrict__ start_pos, int32_t* __restrict__ new_lens,
-    const float* __restrict__ s_tensor_p, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-    int S_max, int32_t* __restrict__ status, const int32_t* __restrict__ block_table, int page_tokens,
-    int max_pages, int num_pages) {
-    const int nblk = D / 16;
-    const int64_t total = (int64_t)B * Hkv * n_new * nblk;
+    const void* __restrict__ x_new, const QShape q, const int32_t* __restrict__ start_pos,
+    int32_t* __restrict__ new_lens, const float* __restrict__ s_tensor_p, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales, int32_t* __restrict__ status, const int32_t* __restrict__ block_table,
+    int page_tokens, int max_pages, int num_pages) {
+    __shared__ QTable tb;
+    const int64_t total = ((int64_t)q.B * q.Hkv * q.n_new) << q.lg_nblk;
     const float st = *s_tensor_p;
     const bool st_ok = st > 0.0f && st <= 3.4028234663852886e38f;  // finite and positive
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int blk = (int)(i % nblk);
-        int64_t r = i / nblk;
-        const int t = (int)(r % n_new);
-        r /= n_new;
-        const int h = (int)(r % Hkv);
-        const int b = (int)(r / Hkv);
-        const bool leader = (t == 0 && h == 0 && blk == 0);
-        if (!st_ok) {
-            if (i == 0) report(status, NVFP4_ERR_NONFINITE);
-            continue;
-        }
-        const int start = start_pos[b];
-        if (start < 0 || (int64_t)start + n_new > S_max) {
-            if (leader) report(status, NVFP4_ERR_CAPACITY);
-            continue;
-        }
-        if (leader && new_lens != nullptr) new_lens[b] = start + n_new;
-        int64_t slot;
-        if (block_table == nullptr) {
-            slot = ((int64_t)b * Hkv + h) * S_max + start + t;
-        } else {
-            const int pos = start + t;
-            const int page = block_table[(int64_t)b * max_pages + pos / page_tokens];
-            if (page < 0 || page >= num_pages) {
-                report(status, NVFP4_ERR_INVALID_ARG);
-                continue;
-            }
-            slot = ((int64_t)page * Hkv + h) * page_tokens + pos % page_tokens;
-        }
-        float v[16];
-        load16<F32>(x_new, (((int64_t)b * n_new + t) * Hkv + h) * D + 16 * blk, v);
-        uint2 packed;
-        const uint32_t sb = quantize_block(v, st, packed);
-        *reinterpret_cast<uint2*>(codes + slot * (D / 2) + 8 * blk) = packed;
-        scales[slot * (D / 16) + blk] = (uint8_t)sb;
+    build_qtable(tb, st);
+    __syncthreads();
+    if (total < (int64_t)INT32_MAX) {
+        for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < (uint32_t)total; i += gridDim.x * blockDim.x)
+            quantize_append_paged_item<F32, uint32_t>(x_new, i, q, start_pos, new_lens, st, st_ok, tb, codes, scales,
+                                                      status, block_table, page_tokens, max_pages, num_pages);
+    } else {
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+             i += (int64_t)gridDim.x * blockDim.x)
+            quantize_append_paged_item<F32, int64_t>(x_new, i, q, start_pos, new_lens, st, st_ok, tb, codes, scales,
+                                                     status, block_table, page_tokens, max_pages, num_pages);
     }
 }
 
@@ -239,49 +370,61 @@ __device__ __forceinline__ uint32_t mxfp4_quantize_block(const float (&a)[16], c
     const uint32_t E = __float_as_uint(amax) >> 23;
     const uint32_t sb = E >= 2u ? E - 2u : 0u;
     const float inv = __uint_as_float((254u - sb) << 23);   // 2^(127 - sb), a normal float
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    // two elements per hardware conversion (finite inputs: the rule of
+    // e2m1_from_float)
+    uint32_t by[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        w[i / 8] |= e2m1_from_float(__fmul_rn(a[i], inv)) << (4 * (i % 8));
-        w[2 + i / 8] |= e2m1_from_float(__fmul_rn(b[i], inv)) << (4 * (i % 8));
+    for (int k = 0; k < 8; ++k) {
+        by[k] = e2m1x2_from_floats(__fmul_rn(a[2 * k], inv), __fmul_rn(a[2 * k + 1], inv));
+        by[8 + k] = e2m1x2_from_floats(__fmul_rn(b[2 * k], inv), __fmul_rn(b[2 * k + 1], inv));
     }
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        w[j] = __byte_perm(by[4 * j] | (by[4 * j + 1] << 8), by[4 * j + 2] | (by[4 * j + 3] << 8), 0x5410);
     packed = make_uint4(w[0], w[1], w[2], w[3]);
     return sb;
 }
 
+template <bool F32, typename I>
+__device__ __forceinline__ void mxfp4_quantize_append_item(
+    const void* __restrict__ x_new, I i, const QShape& q, const int32_t* __restrict__ start_pos,
+    int32_t* __restrict__ new_lens, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+    int32_t* __restrict__ status) {
+    const QItem it = decode_item(q, i);
+    const bool leader = (it.t == 0 && it.h == 0 && it.blk == 0);
+    const int start = start_pos[it.b];
+    if (start < 0 || (int64_t)start + q.n_new > q.S_max) {
+        if (leader) report(status, NVFP4_ERR_CAPACITY);
+        return;
+    }
+    if (leader && new_lens != nullptr) new_lens[it.b] = start + q.n_new;
+    const int64_t elem = (int64_t)i * 32;
+    float va[16], vb[16];
+    load16<F32>(x_new, elem, va);
+    load16<F32>(x_new, elem + 16, vb);
+    uint4 packed;
+    bool bad;
+    const uint32_t sb = mxfp4_quantize_block(va, vb, packed, bad);
+    if (bad) report(status, NVFP4_ERR_NONFINITE);
+    const int64_t slot = ((int64_t)it.b * q.Hkv + it.h) * q.S_max + start + it.t;
+    *reinterpret_cast<uint4*>(codes + slot * (q.D / 2) + 16 * it.blk) = packed;
+    scales[slot * (q.D / 32) + it.blk] = (uint8_t)sb;
+}
+
 template <bool F32>
 __global__ void __launch_bounds__(256) mxfp4_quantize_append_kernel(
-    const void* __restrict__ x_new, int B, int n_new, int Hkv, int D,
-    const int32_t* __restrict__ start_pos, int32_t* __restrict__ new_lens, uint8_t* __restrict__ codes,
-    uint8_t* __restrict__ scales, int S_max, int32_t* __restrict__ status) {
-    const int nblk = D / 32;
-    const int64_t total = (int64_t)B * Hkv * n_new * nblk;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int blk = (int)(i % nblk);
-        int64_t r = i / nblk;
-        const int t = (int)(r % n_new);
-        r /= n_new;
-        const int h = (int)(r % Hkv);
-        const int b = (int)(r / Hkv);
-        const bool leader = (t == 0 && h == 0 && blk == 0);
-        const int start = start_pos[b];
-        if (start < 0 || (int64_t)start + n_new > S_max) {
-            if (leader) report(status, NVFP4_ERR_CAPACITY);
-            continue;
-        }
-        if (leader && new_lens != nullptr) new_lens[b] = start + n_new;
-        const int64_t elem = (((int64_t)b * n_new + t) * Hkv + h) * D + 32 * blk;
-        float va[16], vb[16];
-        load16<F32>(x_new, elem, va);
-        load16<F32>(x_new, elem + 16, vb);
-        uint4 packed;
-        bool bad;
-        const uint32_t sb = mxfp4_quantize_block(va, vb, packed, bad);
-        if (bad) report(status, NVFP4_ERR_NONFINITE);
-        const int64_t slot = ((int64_t)b * Hkv + h) * S_max + start + t;
-        *reinterpret_cast<uint4*>(codes + slot * (D / 2) + 16 * blk) = packed;
-        scales[slot * (D / 32) + blk] = (uint8_t)sb;
+    const void* __restrict__ x_new, const QShape q, const int32_t* __restrict__ start_pos,
+    int32_t* __restrict__ new_lens, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+    int32_t* __restrict__ status) {
+    const int64_t total = ((int64_t)q.B * q.Hkv * q.n_new) << q.lg_nblk;
+    if (total < (int64_t)INT32_MAX) {
+        for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < (uint32_t)total; i += gridDim.x * blockDim.x)
+            mxfp4_quantize_append_item<F32, uint32_t>(x_new, i, q, start_pos, new_lens, codes, scales, status);
+    } else {
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+             i += (int64_t)gridDim.x * blockDim.x)
+            mxfp4_quantize_append_item<F32, int64_t>(x_new, i, q, start_pos, new_lens, codes, scales, status);
     }
 }
 
@@ -295,14 +438,13 @@ cudaError_t launch_mxfp4_quantize_append(const void* x_new, bool f32, int n_new,
     int64_t grid = (total + threads - 1) / threads;
     const int64_t cap = 16L * device_sm_count();
     if (grid > cap) grid = cap;
+    const QShape q = make_qshape(pl.B, n_new, pl.H_kv, pl.D, pl.S_max, 32);
     if (f32)
         mxfp4_quantize_append_kernel<true><<<(int)grid, threads, 0, stream>>>(
-            x_new, pl.B, n_new, pl.H_kv, pl.D, d_start_pos, d_new_lens, pl.codes, pl.scales, pl.S_max,
-            d_status);
+            x_new, q, d_start_pos, d_new_lens, pl.codes, pl.scales, d_status);
     else
         mxfp4_quantize_append_kernel<false><<<(int)grid, threads, 0, stream>>>(
-            x_new, pl.B, n_new, pl.H_kv, pl.D, d_start_pos, d_new_lens, pl.codes, pl.scales, pl.S_max,
-            d_status);
+            x_new, q, d_start_pos, d_new_lens, pl.codes, pl.scales, d_status);
     return cudaGetLastError();
 }
 
@@ -318,14 +460,15 @@ cudaError_t launch_quantize_append_kv(const void* x_k, const void* x_v, bool f32
     const int64_t cap = 8L * device_sm_count();
     if (grid > cap) grid = cap;
     const dim3 g((unsigned)grid, 2);
+    const QShape q = make_qshape(pk.B, n_new, pk.H_kv, pk.D, pk.S_max, 16);
     if (f32)
         quantize_append_kv_kernel<true><<<g, threads, 0, stream>>>(
-            x_k, x_v, pk.B, n_new, pk.H_kv, pk.D, d_start_pos, d_new_lens, d_st_k, d_st_v, pk.codes,
-            pk.scales, pv.codes, pv.scales, pk.S_max, d_status);
+            x_k, x_v, q, d_start_pos, d_new_lens, d_st_k, d_st_v, pk.codes, pk.scales, pv.codes, pv.scales,
+            d_status);
     else
         quantize_append_kv_kernel<false><<<g, threads, 0, stream>>>(
-            x_k, x_v, pk.B, n_new, pk.H_kv, pk.D, d_start_pos, d_new_lens, d_st_k, d_st_v, pk.codes,
-            pk.scales, pv.codes, pv.scales, pk.S_max, d_status);
+            x_k, x_v, q, d_start_pos, d_new_lens, d_st_k, d_st_v, pk.codes, pk.scales, pv.codes, pv.scales,
+            d_status);
     return cudaGetLastError();
 }
 
@@ -339,14 +482,13 @@ cudaError_t launch_quantize_append(const void* x_new, bool f32, int n_new,
     int64_t grid = (total + threads - 1) / threads;
     const int64_t cap = 16L * device_sm_count();
     if (grid > cap) grid = cap;
+    const QShape q = make_qshape(pl.B, n_new, pl.H_kv, pl.D, pl.S_max, 16);
     if (f32)
         quantize_append_kernel<true><<<(int)grid, threads, 0, stream>>>(
-            x_new, pl.B, n_new, pl.H_kv, pl.D, d_start_pos, d_new_lens, d_s_tensor, pl.codes,
-            pl.scales, pl.S_max, d_status, nullptr, 0, 0, 0);
+            x_new, q, d_start_pos, d_new_lens, d_s_tensor, pl.codes, pl.scales, d_status, nullptr, 0, 0, 0);
     else
         quantize_append_kernel<false><<<(int)grid, threads, 0, stream>>>(
-            x_new, pl.B, n_new, pl.H_kv, pl.D, d_start_pos, d_new_lens, d_s_tensor, pl.codes,
-            pl.scales, pl.S_max, d_status, nullptr, 0, 0, 0);
+            x_new, q, d_start_pos, d_new_lens, d_s_tensor, pl.codes, pl.scales, d_status, nullptr, 0, 0, 0);
     return cudaGetLastError();
 }
 
@@ -361,14 +503,15 @@ cudaError_t launch_quantize_append_paged(const void* x_new, bool f32, int n_new,
     const int64_t cap = 16L * device_sm_count();
     if (grid > cap) grid = cap;
     const int S_max = pp.max_pages * pp.page_tokens;   // fits: checked by the caller
+    const QShape q = make_qshape(pp.B, n_new, pp.H_kv, pp.D, S_max, 16);
     if (f32)
         quantize_append_kernel<true><<<(int)grid, threads, 0, stream>>>(
-            x_new, pp.B, n_new, pp.H_kv, pp.D, d_start_pos, d_new_lens, d_s_tensor, pp.codes,
-            pp.scales, S_max, d_status, pp.block_table, pp.page_tokens, pp.max_pages, pp.num_pages);
+            x_new, q, d_start_pos, d_new_lens, d_s_tensor, pp.codes, pp.scales, d_status, pp.block_table,
+            pp.page_tokens, pp.max_pages, pp.num_pages);
     else
         quantize_append_kernel<false><<<(int)grid, threads, 0, stream>>>(
-            x_new, pp.B, n_new, pp.H_kv, pp.D, d_start_pos, d_new_lens, d_s_tensor, pp.codes,
-            pp.scales, S_max, d_status, pp.block_table, pp.page_tokens, pp.max_pages, pp.num_pages);
+            x_new, q, d_start_pos, d_new_lens, d_s_tensor, pp.codes, pp.scales, d_status, pp.block_table,
+            pp.page_tokens, pp.max_pages, pp.num_pages);
     return cudaGetLastError();
 }
 
@@ -378,9 +521,46 @@ cudaError_t launch_quantize_append_paged(const void* x_new, bool f32, int n_new,
 // scale (128 x 8 bytes); each thread then turns one 16-element block into 16
 // FP8 bytes with two table words and byte permutes.
 // ---------------------------------------------------------------------------
+template <typename I>
+__device__ __forceinline__ void dequant_fp8_item(I i, const uint8_t* __restrict__ codes,
+                                                 const uint8_t* __restrict__ scales, int Hkv, int S_max, int D,
+                                                 int lg_nblk, const FastDiv& fd_smax, const FastDiv& fd_hkv,
+                                                 const int32_t* __restrict__ seq_lens, const uint2* lut,
+                                                 uint8_t* __restrict__ out, int32_t* __restrict__ status) {
+    const int blk = (int)(i & (I)((1 << lg_nblk) - 1));
+    const I slot = i >> lg_nblk;                         // (b * Hkv + h) * S_max + t
+    int t, b;
+    bool h0;
+    if constexpr (sizeof(I) == 4) {
+        const uint32_t bh = fd_smax.div((uint32_t)slot);
+        t = (int)((uint32_t)slot - bh * (uint32_t)S_max);
+        b = (int)fd_hkv.div(bh);
+        h0 = bh == (uint32_t)b * (uint32_t)Hkv;
+    } else {
+        t = (int)(slot % S_max);
+        const int64_t bh = slot / S_max;
+        b = (int)(bh / Hkv);
+        h0 = bh % Hkv == 0;
+    }
+    int L = seq_lens[b];
+    if (L > S_max || L < 0) {
+        if (t == 0 && blk == 0 && h0) report(status, NVFP4_ERR_CAPACITY);
+        L = L < 0 ? 0 : S_max;
+    }
+    if (t >= L) return;
+    const int nblk = 1 << lg_nblk;
+    const uint2 c = __ldg(reinterpret_cast<const uint2*>(codes + (int64_t)slot * (D / 2) + 8 * blk));
+    const uint2 l = lut[scales[(int64_t)slot * nblk + blk] & 0x7F];
+    uint4 o;
+    dequant_word(c.x, l.x, l.y, o.x, o.y);
+    dequant_word(c.y, l.x, l.y, o.z, o.w);
+    *reinterpret_cast<uint4*>(out + (int64_t)slot * D + 16 * blk) = o;
+}
+
 __global__ void __launch_bounds__(256) dequant_fp8_kernel(
     const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales, int B, int Hkv,
-    int S_max, int D, const float* __restrict__ s_tensor_p, const int32_t* __restrict__ seq_lens,
+    int S_max, int D, int lg_nblk, const FastDiv fd_smax, const FastDiv fd_hkv,
+    const float* __restrict__ s_tensor_p, const int32_t* __restrict__ seq_lens,
     uint8_t* __restrict__ out, int32_t* __restrict__ status) {
     __shared__ uint2 lut[128];
     const float st = *s_tensor_p;
@@ -388,26 +568,16 @@ __global__ void __launch_bounds__(256) dequant_fp8_kernel(
     if (blockIdx.x == 0 && threadIdx.x == 0 && !(st > 0.0f && st <= 3.4028234663852886e38f))
         report(status, NVFP4_ERR_NONFINITE);
     __syncthreads();
-    const int nblk = D / 16;
-    const int64_t total = (int64_t)B * Hkv * S_max * nblk;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int blk = (int)(i % nblk);
-        const int64_t slot = i / nblk;                       // (b * Hkv + h) * S_max + t
-        const int t = (int)(slot % S_max);
-        const int b = (int)(slot / S_max / Hkv);
-        int L = seq_lens[b];
-        if (L > S_max || L < 0) {
-            if (t == 0 && blk == 0 && (slot / S_max) % Hkv == 0) report(status, NVFP4_ERR_CAPACITY);
-            L = L < 0 ? 0 : S_max;
-        }
-        if (t >= L) continue;
-        const uint2 c = __ldg(reinterpret_cast<const uint2*>(codes + slot * (D / 2) + 8 * blk));
-        const uint2 l = lut[scales[slot * nblk + blk] & 0x7F];
-        uint4 o;
-        dequant_word(c.x, l.x, l.y, o.x, o.y);
-        dequant_word(c.y, l.x, l.y, o.z, o.w);
-        *reinterpret_cast<uint4*>(out + slot * D + 16 * blk) = o;
+    const int64_t total = ((int64_t)B * Hkv * S_max) << lg_nblk;
+    if (total < (int64_t)INT32_MAX) {
+        for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < (uint32_t)total; i += gridDim.x * blockDim.x)
+            dequant_fp8_item<uint32_t>(i, codes, scales, Hkv, S_max, D, lg_nblk, fd_smax, fd_hkv, seq_lens, lut,
+                                       out, status);
+    } else {
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+             i += (int64_t)gridDim.x * blockDim.x)
+            dequant_fp8_item<int64_t>(i, codes, scales, Hkv, S_max, D, lg_nblk, fd_smax, fd_hkv, seq_lens, lut,
+                                      out, status);
     }
 }
 
@@ -418,11 +588,13 @@ cudaError_t launch_dequant_fp8(const nvfp4_kv_plane& pl, const float* d_s_tensor
     if (total == 0) return cudaSuccess;
     const int threads = 256;
     int64_t grid = (total + threads - 1) / threads;
-    const int64_t cap = 4L * device_sm_count();
+    const int64_t cap = 8L * device_sm_count();
     if (grid > cap) grid = cap;
-    dequant_fp8_kernel<<<(int)grid, threads, 0, stream>>>(pl.codes, pl.scales, pl.B, pl.H_kv,
-                                                          pl.S_max, pl.D, d_s_tensor, d_seq_lens,
-                                                          out, d_status);
+    int lg = 0;
+    while ((16 << lg) < pl.D) ++lg;
+    dequant_fp8_kernel<<<(int)grid, threads, 0, stream>>>(pl.codes, pl.scales, pl.B, pl.H_kv, pl.S_max, pl.D, lg,
+                                                          FastDiv((uint32_t)pl.S_max), FastDiv((uint32_t)pl.H_kv),
+                                                          d_s_tensor, d_seq_lens, out, d_status);
     return cudaGetLastError();
 }
 

@@ -180,4 +180,25 @@ def special_blocks(D: int = 128) -> torch.Tensor:
     r = torch.full((D,), 1e-30); r[::3] = -2e-38; rows.append(r)
     r = torch.linspace(-50.0, 50.0, D); rows.append(r)
     r = torch.linspace(-1e4, 3e4, D); rows.append(r)
+    # one float either side of every grid midpoint, in blocks whose amax is 6
+    # (with s_tensor = 1 the block's divisor is exactly 1)
+    mids = torch.tensor([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    below = torch.nextafter(mids, torch.zeros(7))
+    above = torch.nextafter(mids, torch.full((7,), 8.0))
+    blk = torch.cat([below, above, torch.tensor([6.0, -6.0])])
+    r = torch.cat([blk, -blk] * (D // 32)); rows.append(r)
+    # small values of both signs that round to a signed zero or the first code
+    r = torch.tensor([-1e-3, 1e-3, -0.2, 0.2, -0.26, 0.26, -0.0, 6.0] * (D // 8)); rows.append(r)
     return torch.stack(rows)
+
+
+def nonfinite_blocks(D: int = 128) -> torch.Tensor:
+    """Token rows [n][D] with a NaN or an infinity inside blocks of ordinary
+    values (the quantizer's path for blocks it cannot divide by correction)."""
+    r = torch.linspace(-3.0, 3.0, D)
+    r[5] = float("nan")
+    r[40] = float("inf")
+    r[41] = -float("inf")
+    r2 = torch.linspace(-1.0, 1.0, D)
+    r2[16:32] = float("nan")
+    return torch.stack([r, r2])

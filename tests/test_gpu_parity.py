@@ -121,6 +121,44 @@ def test_special_blocks_bit_exact(nv):
             np.testing.assert_array_equal(plane.scales[0, 0, :n].cpu().numpy(), ks[0, 0, :n])
 
 
+def test_nonfinite_blocks_bit_exact(nv):
+    # NaN and infinite elements: no status (the append does not check its
+    # input), codes and scales as the oracle's -- a NaN element gives code 0x7
+    rows = synthetic.nonfinite_blocks(128)
+    x = rows.view(1, rows.shape[0], 1, 128).contiguous()
+    for st in (np.float32(1.0), np.float32(0.01)):
+        plane = nv.KVPlane.allocate(1, 1, 16, 128)
+        s = torch.tensor([st], device="cuda")
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        nv.nvfp4_kv_quantize_append(x.cuda(), torch.zeros(1, dtype=torch.int32, device="cuda"), s, plane,
+                                    status=status)
+        torch.cuda.synchronize()
+        assert status.item() == 0
+        kc, ks = oracle.new_planes(1, 1, 16, 128)
+        assert oracle.quantize_append(x.numpy(), np.zeros(1, np.int32), st, kc, ks) == 0
+        n = rows.shape[0]
+        np.testing.assert_array_equal(plane.codes[0, 0, :n].cpu().numpy(), kc[0, 0, :n])
+        np.testing.assert_array_equal(plane.scales[0, 0, :n].cpu().numpy(), ks[0, 0, :n])
+
+
+def test_quantize_wide_range_f32_bit_exact(nv):
+    # fp32 inputs over 60 binades and tensor scales over 40: the division by
+    # correction and the hardware E2M1 conversion give the oracle's codes
+    g = torch.Generator().manual_seed(2024)
+    n_tok, H, D = 512, 4, 128
+    mag = torch.exp2(torch.empty(n_tok, H, D).uniform_(-30.0, 30.0, generator=g))
+    sign = torch.where(torch.rand(n_tok, H, D, generator=g) < 0.5, -1.0, 1.0)
+    x = (mag * sign).view(1, n_tok, H, D).contiguous()
+    for st in (np.float32(3.7e-9), np.float32(0.0123), np.float32(1.0), np.float32(2.9e3), np.float32(6.1e5)):
+        plane = nv.KVPlane.allocate(1, H, n_tok, D)
+        s = torch.tensor([st], device="cuda")
+        nv.nvfp4_kv_quantize_append(x.cuda(), torch.zeros(1, dtype=torch.int32, device="cuda"), s, plane)
+        kc, ks = oracle.new_planes(1, H, n_tok, D)
+        assert oracle.quantize_append(x.numpy(), np.zeros(1, np.int32), st, kc, ks) == 0
+        np.testing.assert_array_equal(plane.codes.cpu().numpy(), kc)
+        np.testing.assert_array_equal(plane.scales.cpu().numpy(), ks)
+
+
 @pytest.mark.parametrize("D", [64, 128])
 def test_dequant_random_planes_bit_exact(nv, D):
     B, H, S = 2, 3, 64
