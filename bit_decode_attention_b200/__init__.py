@@ -29,6 +29,7 @@ __all__ = [
     "nvfp4_version", "NativeError", "nvfp4_decode_attention_noalloc",
     "mxfp4_cache_bytes", "mxfp4_kv_quantize_append",
     "PagedKVPlane", "nvfp4_kv_quantize_append_paged", "nvfp4_decode_attention_paged",
+    "nvfp4_prefill_attention",
 ]
 
 
@@ -229,6 +230,25 @@ def new_workspace(B: int, H_q: int, H_kv: int, D: int, device="cuda") -> torch.T
     if n == 0:
         raise ValueError("unsupported attention shape")
     return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def nvfp4_prefill_attention(q: torch.Tensor, k: KVPlane, v: KVPlane, s_tensor_k: torch.Tensor,
+                            s_tensor_v: torch.Tensor, start_pos: torch.Tensor, softmax_scale: float = 0.0,
+                            out: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                            stream=None) -> torch.Tensor:
+    """Causal attention of a prompt chunk over the NVFP4 cache (the chunk's K/V
+    already appended at start_pos); q [B][C][H_q][128] -> fp32 [B][C][H_q][128]."""
+    _need_cuda(q, s_tensor_k, s_tensor_v, start_pos, out, status)
+    B, C, H_q, D = q.shape
+    if out is None:
+        out = torch.empty(B, C, H_q, D, dtype=torch.float32, device=q.device)
+    kp, vp = k.struct(), v.struct()
+    st = _native.lib().nvfp4_prefill_attention(
+        _ptr(q), _dtype_code(q), C, H_q, ctypes.byref(kp), ctypes.byref(vp), _ptr(s_tensor_k),
+        _ptr(s_tensor_v), _ptr(start_pos), ctypes.c_float(softmax_scale), _ptr(out), _ptr(status),
+        _stream(stream))
+    _native.check("nvfp4_prefill_attention", st)
+    return out
 
 
 def nvfp4_decode_attention(q: torch.Tensor, k: KVPlane, v: KVPlane, s_tensor_k: torch.Tensor,

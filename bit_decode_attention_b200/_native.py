@@ -40,6 +40,7 @@ EXPORTS = (
     "nvfp4_decode_attention_paged",
     "nvfp4_decode_attention_append",
     "nvfp4_set_wait_limit",
+    "nvfp4_prefill_attention",
 )
 
 
@@ -127,6 +128,8 @@ def lib():
     L.nvfp4_decode_attention_append.restype = i32
     L.nvfp4_set_wait_limit.argtypes = [i64]
     L.nvfp4_set_wait_limit.restype = None
+    L.nvfp4_prefill_attention.argtypes = [vp, i32, i32, i32, plane_p, plane_p, vp, vp, vp, f32, vp, vp, vp]
+    L.nvfp4_prefill_attention.restype = i32
     _lib = L
     return L
 

@@ -404,4 +404,30 @@ nvfp4_status nvfp4_decode_attention_paged(const void* q, nvfp4_dtype q_dtype, in
                          workspace_bytes, d_status, stream);
 }
 
+nvfp4_status nvfp4_prefill_attention(const void* q, nvfp4_dtype q_dtype, int C, int H_q,
+                                     const nvfp4_kv_plane* k, const nvfp4_kv_plane* v,
+                                     const float* d_s_tensor_k, const float* d_s_tensor_v,
+                                     const int32_t* d_start_pos, float softmax_scale, float* out,
+                                     int32_t* d_status, nvfp4_stream_t stream) {
+    if (!plane_ok(k) || !plane_ok(v)) return NVFP4_ERR_INVALID_ARG;
+    if (k->B != v->B || k->H_kv != v->H_kv || k->S_max != v->S_max || k->D != v->D)
+        return NVFP4_ERR_INVALID_ARG;
+    if (q_dtype != NVFP4_IN_BF16 && q_dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
+    if (C < 0 || H_q <= 0 || (H_q % k->H_kv) != 0) return NVFP4_ERR_INVALID_ARG;
+    if (d_s_tensor_k == nullptr || d_s_tensor_v == nullptr || d_start_pos == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!(std::isfinite(softmax_scale)) || softmax_scale < 0.0f) return NVFP4_ERR_INVALID_ARG;
+    // the tensor-core prefill takes bf16 queries (exact in its f16 operand);
+    // an fp32 query would need a second f16 term and its shared memory
+    if (k->D != 128 || H_q / k->H_kv > 128 || q_dtype != NVFP4_IN_BF16) return NVFP4_ERR_UNSUPPORTED;
+    if (k->B == 0 || C == 0) return NVFP4_OK;
+    if (q == nullptr || out == nullptr || !aligned16(q) || !aligned16(out)) return NVFP4_ERR_INVALID_ARG;
+    const int g = H_q / k->H_kv, cq = 128 / g;
+    if ((int64_t)k->B * k->H_kv * ((C + cq - 1) / cq) > (int64_t)INT32_MAX) return NVFP4_ERR_UNSUPPORTED;
+    return from_cuda(launch_prefill_tc(q, q_dtype == NVFP4_IN_F32, C, H_q, *k, *v, d_s_tensor_k, d_s_tensor_v,
+                                       d_start_pos, softmax_scale, out, d_status,
+                                       g_wait_polls.load(std::memory_order_relaxed),
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -95,6 +95,12 @@ struct AttnLaunch {
 
 cudaError_t launch_decode_attention(const AttnLaunch& a, cudaStream_t stream);
 
+// chunked-prefill attention on the tensor cores (head_dim 128, contiguous planes)
+cudaError_t launch_prefill_tc(const void* q, bool q_f32, int C, int H_q, const nvfp4_kv_plane& k,
+                              const nvfp4_kv_plane& v, const float* d_st_k, const float* d_st_v,
+                              const int32_t* d_start, float softmax_scale, float* out, int32_t* d_status,
+                              uint32_t wait_polls, cudaStream_t stream);
+
 // workspace layout of nvfp4_decode_attention for one shape
 struct AttnWorkspace {
     size_t counters_bytes;  // B * H_kv int32, padded to 256 bytes

@@ -260,6 +260,33 @@ nvfp4_status nvfp4_decode_attention(const void* q, nvfp4_dtype q_dtype, int H_q,
                                     float* out, void* workspace, size_t workspace_bytes,
                                     int32_t* d_status, nvfp4_stream_t stream);
 
+/* Chunked-prefill attention over the cache ([NVFP4-KV] "推論速度": the NVFP4
+ * cache shortens time to first token, the prefill side; "量子化・逆量子化フロー":
+ * attention runs over the cache dequantized to FP8).  A chunk of C prompt
+ * tokens per sequence, already appended to the cache at slots start_pos[b] ..
+ * start_pos[b] + C - 1, attends causally: query i of sequence b sees the
+ * cache tokens t <= start_pos[b] + i.  Runs on the tensor cores (tcgen05,
+ * f16 MMAs with fp32 accumulation; the cache's FP8 values are exact in f16,
+ * and so is a bf16 query after a power-of-two row scaling; the
+ * probabilities enter as two f16 terms, about 22 significant bits).
+ *   q           device [B][C][H_q][128] bf16, 16-byte aligned (fp32 queries:
+ *               NVFP4_ERR_UNSUPPORTED)
+ *   C           chunk length (0: nothing to do)
+ *   H_q         query heads, a multiple of H_kv with H_q / H_kv <= 128
+ *   k, v        contiguous planes of head_dim 128 (other D: NVFP4_ERR_UNSUPPORTED)
+ *   d_start_pos device int32 [B], the chunk's first position per sequence
+ *   softmax_scale  0 selects 1 / sqrt(128)
+ *   out         device float [B][C][H_q][128], overwritten
+ * A sequence with start_pos < 0 or start_pos + C > S_max is skipped and
+ * NVFP4_ERR_CAPACITY goes to *d_status (its output rows are left as they
+ * were); a non-finite or non-positive tensor scale reports
+ * NVFP4_ERR_NONFINITE.  Host errors as for nvfp4_decode_attention. */
+nvfp4_status nvfp4_prefill_attention(const void* q, nvfp4_dtype q_dtype, int C, int H_q,
+                                     const nvfp4_kv_plane* k, const nvfp4_kv_plane* v,
+                                     const float* d_s_tensor_k, const float* d_s_tensor_v,
+                                     const int32_t* d_start_pos, float softmax_scale, float* out,
+                                     int32_t* d_status, nvfp4_stream_t stream);
+
 /* Append one decode token per sequence, then attend over the cache including
  * it, in one call ([NVFP4-KV] "量子化・逆量子化フロー": the new K/V are
  * quantized to NVFP4 as they enter the cache, then FP8 attention runs over

@@ -149,6 +149,13 @@ def queries(w: Workload, stream: int = 0, batch: Optional[int] = None) -> torch.
     return _round_dtype(torch.randn(B, w.Hq, w.D, generator=g), w)
 
 
+def prefill_queries(w: Workload, C: int, stream: int = 0) -> torch.Tensor:
+    """Queries of a C-token prompt chunk ~ N(0,1), fp32 values exactly
+    representable in w.dtype, shape [B][C][Hq][D]."""
+    g = generator(w, stream=300 + stream)
+    return _round_dtype(torch.randn(w.B, C, w.Hq, w.D, generator=g), w)
+
+
 def capacity(max_len: int, extra: int = 0) -> int:
     """Cache capacity S_max for a workload: max_len + extra rounded up to 16."""
     n = max_len + extra

@@ -635,3 +635,70 @@ def test_attention_wait_timeout_reports_and_recovers(nv):
     torch.cuda.synchronize()
     assert status.item() == 0
     assert_attention_close(got.cpu().numpy(), want)
+
+
+# ---- chunked-prefill attention (tensor cores) ----
+def _prefill_case(w, start, C, q_dtype=None):
+    # the cache holds every sequence up to the end of its chunk
+    case = Case(w, lens=[s + C for s in start], q_dtype=q_dtype)
+    q = synthetic.prefill_queries(w, C)
+    if q_dtype is not None and q_dtype != w.dtype:
+        q = q.to(torch.bfloat16 if q_dtype == "bf16" else torch.float32).float()
+    return case, q
+
+
+def _check_prefill(nv, w, start, C, q_dtype=None, softmax_scale=0.0):
+    case, q = _prefill_case(w, start, C, q_dtype)
+    qd = q_dtype or w.dtype
+    start_d = torch.tensor(start, dtype=torch.int32, device="cuda")
+    got = nv.nvfp4_prefill_attention(to_dev(q, qd), case.k, case.v, case.sk, case.sv, start_d,
+                                     softmax_scale=softmax_scale, status=case.status)
+    torch.cuda.synchronize()
+    assert case.status.item() == 0
+    kc, ks, vc, vs = case.oracle_planes()
+    want = oracle.prefill_attention_nvfp4(q.numpy(), kc, ks, vc, vs, case.sk_o, case.sv_o,
+                                          np.array(start, np.int32), softmax_scale)
+    return assert_attention_close(got.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("g,C,start", [(4, 200, [0, 300]), (8, 130, [5, 129]), (1, 300, [77, 0]),
+                                       (16, 40, [1000, 3]), (12, 97, [256, 511])])
+def test_prefill_attention_parity(nv, g, C, start):
+    w = synthetic.shrink(synthetic.get("gqa"), B=len(start), Hkv=2, Hq=2 * g)
+    _check_prefill(nv, w, start, C)
+
+
+def test_prefill_attention_softmax_scale_and_f32_rejected(nv):
+    w = synthetic.shrink(synthetic.get("gqa"), B=2, Hkv=1, Hq=8)
+    _check_prefill(nv, w, [100, 3], 150, softmax_scale=0.05)
+    # fp32 queries are not taken by the tensor-core prefill
+    case, q = _prefill_case(w, [0, 0], 16)
+    start_d = torch.zeros(2, dtype=torch.int32, device="cuda")
+    with pytest.raises(nv.NativeError):
+        nv.nvfp4_prefill_attention(q.cuda(), case.k, case.v, case.sk, case.sv, start_d)
+
+
+def test_prefill_attention_2048_chunk_group12(nv):
+    # the large-MoE shape's chunk: 2048 queries x a GQA group of 12, after
+    # 1024 cached tokens (two KV heads keep the oracle to seconds)
+    w = synthetic.shrink(synthetic.get("moe128k"), B=1, Hkv=2, Hq=24)
+    _check_prefill(nv, w, [1024], 2048)
+
+
+def test_prefill_attention_capacity_and_empty(nv):
+    w = synthetic.shrink(synthetic.get("gqa"), B=2, Hkv=1, Hq=4)
+    case, q = _prefill_case(w, [0, 0], 64)
+    start_d = torch.tensor([0, case.S_max - 10], dtype=torch.int32, device="cuda")
+    out = torch.full((2, 64, 4, 128), 7.0, device="cuda")
+    nv.nvfp4_prefill_attention(to_dev(q, w.dtype), case.k, case.v, case.sk, case.sv, start_d, out=out,
+                               status=case.status)
+    torch.cuda.synchronize()
+    assert case.status.item() == nv.NVFP4_ERR_CAPACITY
+    assert torch.all(out[1] == 7.0).item()              # the over-long sequence is skipped
+    kc, ks, vc, vs = case.oracle_planes(0)
+    want = oracle.prefill_attention_nvfp4(q[:1].numpy(), kc, ks, vc, vs, case.sk_o, case.sv_o,
+                                          np.zeros(1, np.int32))
+    assert_attention_close(out[:1].cpu().numpy(), want)
+    # an empty chunk is a no-op
+    empty = torch.empty(2, 0, 4, 128, device="cuda", dtype=torch.bfloat16)
+    nv.nvfp4_prefill_attention(empty, case.k, case.v, case.sk, case.sv, start_d)
