@@ -52,6 +52,7 @@ DTYPE = ("nvfp4 storage (e2m1 codes + e4m3 block scales + f32 tensor scale); e4m
          "operands (K, V exact FP8; q as 2 e4m3 terms, P as 3 e4m3 terms); f32 accumulate")
 DEFAULT_WORKLOAD = "ragged"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 ATTN_SOURCES = ["bit_decode_attention_b200/csrc/nvfp4kv_decode_attention_tc.cu",
                 "bit_decode_attention_b200/csrc/nvfp4kv_attention_common.cuh",
                 "bit_decode_attention_b200/csrc/nvfp4kv_tcgen05.cuh",
@@ -675,6 +676,46 @@ def aux_attention(name, w, l2, steps, world, peak, peak_kind, with_append=False,
     return line
 
 
+def aux_prefill(w, C=2048, reps=5):
+    """Chunked-prefill attention on the tensor cores: the last C-token chunk of
+    the workload's context (queries at positions L - C .. L - 1 over the whole
+    cache), timed with CUDA events; tensor roofline in algorithmic FLOPs (the
+    visible query-token pairs, 2 matmuls x 2 FLOP x head_dim)."""
+    import bit_decode_attention_b200 as nv
+    wl = DecodeWorkload(w, 1, with_append=False)
+    L = wl.lens0[0]
+    start = L - C
+    g = torch.Generator().manual_seed(31)
+    q = torch.randn(w.B, C, w.Hq, w.D, generator=g).to(torch.bfloat16).cuda()
+    start_d = torch.full((w.B,), start, dtype=torch.int32, device="cuda")
+    out = torch.empty(w.B, C, w.Hq, w.D, dtype=torch.float32, device="cuda")
+    run = lambda: nv.nvfp4_prefill_attention(q, wl.k[0], wl.v[0], wl.sk, wl.sv, start_d, out=out,
+                                             status=wl.status)
+    ms = time_events(run, reps=reps, warm=2)
+    pairs = w.B * w.Hq * (C * start + C * (C + 1) // 2)
+    flops = 4.0 * w.D * pairs
+    tflops = flops / (ms / 1e3) / 1e12
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except Exception:
+        pass
+    peak, kind = (float(peaks["bf16_tflops"]), "measured bf16 dense (burst)") if "bf16_tflops" in peaks \
+        else (FALLBACK_BF16_TFLOPS, "fallback")
+    line = {"workload": "%s: prefill chunk C=%d at positions %d..%d, B%d Hq%d Hkv%d D%d" %
+                        (w.name, C, start, L - 1, w.B, w.Hq, w.Hkv, w.D),
+            "launch_ms": ms, "achieved_tflops": tflops,
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tflops / peak, "peak_kind": kind, "traffic": None,
+                         "note": "kind::f16 MMAs (the bf16 rate); P.V runs twice (two-term P), so the "
+                                 "tensor pipe executes 1.5x the algorithmic FLOPs"},
+            "gpu_launches": reps, "device_status": wl.status.item()}
+    del wl, q, out
+    torch.cuda.empty_cache()
+    return line
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -746,6 +787,7 @@ def main():
                                         with_append=True)
         aux["gqa_paged_attention"] = aux_attention("gqa_paged", synthetic.get("gqa"), l2, n_aux, world,
                                                    peak, peak_kind, paged=True)
+        aux["moe128k_prefill_attention"] = aux_prefill(synthetic.get("moe128k"))
         aux["gqa_attention_hot_l2"] = aux_attention(
             "gqa_hot", synthetic.get("gqa"), l2, n_aux, world, peak, peak_kind, replicas=1,
             label_extra=" -- HOT L2: one cache (38 MB < L2) re-read every step, not a DRAM number")
