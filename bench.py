@@ -716,6 +716,25 @@ def aux_prefill(w, C=2048, reps=5):
     return line
 
 
+def profile_launches(name):
+    """A few launches of one kernel for an ncu capture (nothing timed)."""
+    import bit_decode_attention_b200 as nv
+    if name == "prefill":
+        w = synthetic.shrink(synthetic.get("moe128k"), L=16384)
+        wl = DecodeWorkload(w, 1, with_append=False)
+        C, start = 2048, wl.lens0[0] - 2048
+        q = torch.randn(w.B, C, w.Hq, w.D, generator=torch.Generator().manual_seed(31)).to(torch.bfloat16).cuda()
+        start_d = torch.full((w.B,), start, dtype=torch.int32, device="cuda")
+        for _ in range(3):
+            nv.nvfp4_prefill_attention(q, wl.k[0], wl.v[0], wl.sk, wl.sv, start_d, status=wl.status)
+    else:
+        wl = DecodeWorkload(synthetic.get(name), 2, with_append=False)
+        for j in range(4):
+            wl.step(j)
+    torch.cuda.synchronize()
+    print("profile launches done, device status", wl.status.item())
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -726,7 +745,14 @@ def main():
     ap.add_argument("--no-aux", action="store_true", help="skip the other workloads' lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=500)
+    ap.add_argument("--profile", metavar="WORKLOAD",
+                    help="for ncu captures: build WORKLOAD's cache (2 replicas), run 4 attention "
+                         "launches (plus the split-K merges) and exit; 'prefill' runs 3 prefill "
+                         "launches (B1 Hq96 Hkv8, a 2048-token chunk after 14336 cached tokens)")
     args = ap.parse_args()
+    if args.profile:
+        profile_launches(args.profile)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     rank, world, local_rank = env_rank()
