@@ -56,7 +56,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 ATTN_SOURCES = ["bit_decode_attention_b200/csrc/nvfp4kv_decode_attention_tc.cu",
                 "bit_decode_attention_b200/csrc/nvfp4kv_attention_common.cuh",
                 "bit_decode_attention_b200/csrc/nvfp4kv_tcgen05.cuh",
-                "bit_decode_attention_b200/csrc/nvfp4kv_device.cuh"]
+                "bit_decode_attention_b200/csrc/nvfp4kv_device.cuh",
+                "bit_decode_attention_b200/csrc/nvfp4kv_pipeline.cuh"]
 GEN_SEQS = 16          # sequences drawn per host block when generating prefill inputs
 
 
