@@ -29,7 +29,7 @@ __all__ = [
     "nvfp4_version", "NativeError", "nvfp4_decode_attention_noalloc",
     "mxfp4_cache_bytes", "mxfp4_kv_quantize_append",
     "PagedKVPlane", "nvfp4_kv_quantize_append_paged", "nvfp4_decode_attention_paged",
-    "nvfp4_prefill_attention",
+    "nvfp4_prefill_attention", "nvfp4_decode_attention_append", "nvfp4_set_wait_limit",
 ]
 
 
