@@ -63,6 +63,11 @@ constexpr int kStages = 4;                            // bulk-copy ring
 constexpr int kBuf = 4;                               // K/S and V^T/P operand buffers
 constexpr int NTERM = 3;                              // E4M3 terms of P
 
+// Hand-offs: every thread that produced (or last read) what a barrier
+// guards fences and arrives on it itself (arrival counts of 128 per group):
+// a per-warp arrival after __syncwarp let the tensor core and the bulk copies
+// race with the other lanes' accesses in the prefill kernel built the same way.
+//
 // warp roles, in warpgroups of four (warp w reaches tensor-memory lanes
 // 32 * (w % 4) .. +31, so every group covers the 128 token lanes):
 //   warps  0- 3, 8-11, 12-15, 16-19  dequant groups 0..3: group i takes the
@@ -541,20 +546,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
     if (warp == kLoadWarp && lane == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.empty[s], 4);
+            mbar_init(&sm.empty[s], 128);
         }
         for (int b = 0; b < kBuf; ++b) {
-            mbar_init(&sm.kfull[b], 4);
+            mbar_init(&sm.kfull[b], 128);
             mbar_init(&sm.qkdone[b], 1);
-            mbar_init(&sm.sempty[b], 4 * n_sgrp);
-            mbar_init(&sm.vfull[b], 4);
-            mbar_init(&sm.pfull[b], 4 * n_sgrp);
+            mbar_init(&sm.sempty[b], 128 * n_sgrp);
+            mbar_init(&sm.vfull[b], 128);
+            mbar_init(&sm.pfull[b], 128 * n_sgrp);
             mbar_init(&sm.pvdone[b], 1);
         }
         mbar_init(&sm.qfull[0], 4 * n_sgrp);
         mbar_init(&sm.qfull[1], 4 * n_sgrp);
         mbar_init(&sm.mma_done, 2);                   // both MMA warps commit
-        mbar_init(&sm.appended, 1);
+        mbar_init(&sm.appended, 32);                  // every lane of the append warp
         fence_mbar_init();
         sm.abort_flag = 0;
         // the first two tiles only: the CTA barrier below waits for this lane;
@@ -706,8 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
         // ================= the fused append's new tokens =================
         if (p.x_k_new != nullptr) {
             append_new_tokens(p, sm.prefix, sm.lens, B, t_begin, t_end, st_k, st_v, lane);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.appended);
+            mbar_arrive(&sm.appended);                 // after this lane's async-proxy fence
         }
     } else if (!is_softmax) {
         // ======== dequant group i: tiles w = i (mod 4), K and V of token t ========
@@ -758,11 +762,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
             for (int j = 0; j < 4; ++j) vc[j] = *reinterpret_cast<const uint4*>(st + OFF_VC + t * kKB + 16 * j);
             tc::tmem_wait_st();
             tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&sm.kfull[i]);                 // Q.K^T of tile w may start
-                mbar_arrive(&sm.empty[i]);                 // the loader may refill stage i
-            }
+            mbar_arrive(&sm.kfull[i]);                     // Q.K^T of tile w may start
+            fence_proxy_async_smem();                      // these ring reads come before the refill
+            mbar_arrive(&sm.empty[i]);                     // the loader may refill stage i
             // P.V of tile w - 4 has read this V^T buffer
             if (w >= 4 && !group_wait(&sm.pvdone[i], ph ^ 1u, poller, gbar, abort_flag, p.status, polls)) break;
 #pragma unroll
@@ -784,8 +786,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
                 }
             }
             fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.vfull[i]);     // P.V of tile w may start
+            mbar_arrive(&sm.vfull[i]);                     // P.V of tile w may start
         }
     } else if (is_softmax && sgrp >= n_sgrp) {
         // a group with padding queries only: nothing to do (its P columns stay
@@ -881,11 +882,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
                     }
                     tc::tmem_wait_ld();
                     tc::fence_before_sync();
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(&sm.sempty[b0]);
-                        if (two) mbar_arrive(&sm.sempty[b1]);
-                    }
+                    mbar_arrive(&sm.sempty[b0]);
+                    if (two) mbar_arrive(&sm.sempty[b1]);
                     const bool live0 = t < valid0, live1 = t < valid1;
 #pragma unroll
                     for (int q = 0; q < NH; ++q) {
@@ -993,11 +991,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_tc_kernel(const 
                     }
                     fence_proxy_async_smem();
                     tc::fence_before_sync();
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(&sm.pfull[b0]);
-                        if (two) mbar_arrive(&sm.pfull[b1]);
-                    }
+                    mbar_arrive(&sm.pfull[b0]);
+                    if (two) mbar_arrive(&sm.pfull[b1]);
                 }
                 any_pv = true;
                 w += two ? 2u : 1u;
