@@ -149,6 +149,24 @@ def test_argument_validation_without_gpu(lib):
         assert ap(*pargs(bp, bp, dev, 1 << 30)) == INVALID
     assert ap(*pargs(pg, pg_other, dev, 1 << 30)) == INVALID     # K and V tables differ
     assert ap(*pargs(pg, pg, dev, 16)) == WS
+    # chunked prefill: head_dim 128 and bf16 queries only; checks before any launch
+    pf = lib.nvfp4_prefill_attention
+    k128, v128 = _plane(B=2, H=2), _plane(B=2, H=2)
+    k64 = _plane(B=2, H=2, D=64)
+    pfa = lambda q, dt, C, hq, kk, vv, st, scale, out: (q, dt, C, hq, ctypes.byref(kk), ctypes.byref(vv), dev,
+                                                        dev, st, ctypes.c_float(scale), out, None, None)
+    UNSUP = _native.NVFP4_ERR_UNSUPPORTED
+    assert pf(*pfa(dev, 0, 16, 3, k128, v128, dev, 0.0, dev)) == INVALID        # H_q % H_kv
+    assert pf(*pfa(dev, 0, 16, 4, k128, v_other, dev, 0.0, dev)) == INVALID     # planes disagree
+    assert pf(*pfa(dev, 0, -1, 4, k128, v128, dev, 0.0, dev)) == INVALID        # negative chunk
+    assert pf(*pfa(dev, 0, 16, 4, k128, v128, None, 0.0, dev)) == INVALID       # no start positions
+    assert pf(*pfa(dev, 0, 16, 4, k128, v128, dev, -1.0, dev)) == INVALID       # softmax scale
+    assert pf(*pfa(dev, 7, 16, 4, k128, v128, dev, 0.0, dev)) == INVALID        # dtype
+    assert pf(*pfa(dev, 1, 16, 4, k128, v128, dev, 0.0, dev)) == UNSUP          # fp32 queries
+    assert pf(*pfa(dev, 0, 16, 4, k64, k64, dev, 0.0, dev)) == UNSUP            # head_dim 64
+    assert pf(*pfa(ctypes.c_void_p(72), 0, 16, 4, k128, v128, dev, 0.0, dev)) == INVALID   # q misaligned
+    assert pf(*pfa(dev, 0, 16, 4, k128, v128, dev, 0.0, None)) == INVALID       # no output
+    assert pf(*pfa(dev, 0, 0, 4, k128, v128, dev, 0.0, dev)) == 0               # empty chunk: no-op
     cal = lib.nvfp4_calib_tensor_scale
     assert cal(dev, 0, -1, dev, None, None) == INVALID
     assert cal(dev, 0, 10, None, None, None) == INVALID
