@@ -196,8 +196,9 @@ nvfp4_status mxfp4_kv_quantize_append(const void* x_new, nvfp4_dtype dtype, int 
                                       const nvfp4_kv_plane* plane, int32_t* d_status,
                                       nvfp4_stream_t stream);
 
-/* nvfp4_kv_quantize_append into a paged plane: the slot of token t of
- * sequence b is found through the block table.  Capacity errors as for
+/* nvfp4_kv_quantize_append into a paged plane ([NVFP4-KV] "学術研究との関連":
+ * PagedAttention's block management combines with the NVFP4 cache): the slot
+ * of token t of sequence b is found through the block table.  Capacity errors as for
  * contiguous planes (start + n_new > max_pages * page_tokens); a block-table
  * entry outside [0, num_pages) skips that token's blocks and reports
  * NVFP4_ERR_INVALID_ARG through *d_status. */
@@ -229,11 +230,14 @@ nvfp4_status nvfp4_kv_dequant_fp8(const nvfp4_kv_plane* plane, const float* d_s_
                                   int32_t* d_status, nvfp4_stream_t stream);
 
 /* Workspace bytes nvfp4_decode_attention needs on the current device for
- * this shape (split-K partial results and per-(sequence, KV head) arrival
- * counters).  Returns 0 for invalid shapes.  The workspace must be
- * zero-filled once after allocation; every completed call leaves its
- * counters at zero again, so it can be reused without clearing.  Calls that
- * share one workspace must not overlap on the GPU. */
+ * this shape: the split-K partial results and per-(sequence, KV head)
+ * arrival counters of the stream-K split ([llama.cpp digest] "CUDA/Vulkan/
+ * HEXAGONの主要バグ修正": the split is sized to the GPU's SM count, so that
+ * no SM idles).  The size depends on the current device's SM count: query
+ * it on the device that will run the calls.  Returns 0 for invalid shapes.
+ * The workspace must be zero-filled once after allocation; every completed
+ * call leaves its counters at zero again, so it can be reused without
+ * clearing.  Calls that share one workspace must not overlap on the GPU. */
 size_t nvfp4_decode_attention_workspace(int B, int H_q, int H_kv, int D);
 
 /* Decode attention over an NVFP4 cache with FP8 dequantization fused in
