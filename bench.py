@@ -88,17 +88,19 @@ def source_digest(paths):
 
 
 def profiled_traffic(name):
-    """DRAM bytes per launch from a committed ncu summary, only while the
-    kernel source still matches the one that was profiled."""
+    """(DRAM bytes per launch from a committed ncu summary, why it is None):
+    the bytes only while the kernel source still matches the one that was
+    profiled."""
     path = os.path.join(ROOT, "profiles", name)
     try:
         with open(path) as f:
             d = json.load(f)
     except Exception:
-        return None
+        return None, "no ncu capture of this workload under profiles/"
     if d.get("source_digest") != source_digest(ATTN_SOURCES):
-        return None
-    return d.get("dram_bytes_per_launch")
+        return None, ("kernel sources changed since the capture in profiles/%s (digest %s); "
+                      "not re-captured" % (name, d.get("source_digest")))
+    return d.get("dram_bytes_per_launch"), None
 
 
 def kv_bytes_per_token(Hkv, D):
@@ -482,16 +484,20 @@ def roofline_block(wl, att_ms, att_n, peak, peak_kind, traffic_name=None):
         return None
     achieved = wl.attention_bytes() / (att_ms / 1e3) / 1e9
     g = wl.w.Hq // wl.w.Hkv
-    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+    traffic, why = profiled_traffic(traffic_name) if traffic_name else (None, "no capture named")
+    block = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak,
             "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
             else "fallback",
-            "traffic": profiled_traffic(traffic_name) if traffic_name else None,
+            "traffic": traffic,
             "kernel": "decode_attention_tc_kernel<%d> + merge_split_units_kernel (tcgen05, head_dim "
                       "128, bf16 queries, GQA group %d)" % (1 if g <= 8 else 2, g),
             "algorithmic_bytes_per_launch": wl.attention_bytes(),
             "launch_ms": att_ms, "launches_sampled": att_n,
             "frac_of_nominal_8tbs": achieved / 8000.0}
+    if why:
+        block["traffic_note"] = why
+    return block
 
 
 def workload_label(w, wl):

@@ -10,12 +10,37 @@
 // E4M3 is the OCP E4M3FN byte: bias 7, largest finite 448, S.1111.111 = NaN.
 #pragma once
 
+#include <cmath>
 #include <cstdint>
 #include <cuda_runtime.h>
 
 #include "../../include/nvfp4kv.h"
 
 namespace nvfp4kv {
+
+// ---------------------------------------------------------------------------
+// Division by a launch-invariant divisor (T. Granlund and P. Montgomery,
+// "Division by Invariant Integers using Multiplication", 1994): for
+// 1 <= d < 2^31 and 0 <= x < 2^31, x / d = (umulhi(x, m) + x) >> l with
+// l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1 (mod 2^32).  A
+// runtime 32-bit division is a software routine of a few dozen instructions;
+// this is two.  (umulhi(x, m) <= x, so the sum stays below 2^32.)
+// ---------------------------------------------------------------------------
+struct FastDiv {
+    uint32_t d, m, l;
+    FastDiv() = default;
+    __host__ explicit FastDiv(uint32_t d_) : d(d_), m(0), l(0) {
+        while ((1ull << l) < d) ++l;
+        m = (uint32_t)((((1ull << 32) * ((1ull << l) - d)) / d + 1) & 0xFFFFFFFFull);
+    }
+    __host__ __device__ __forceinline__ uint32_t div(uint32_t x) const {
+#ifdef __CUDA_ARCH__
+        return (__umulhi(x, m) + x) >> l;
+#else
+        return (uint32_t)((((uint64_t)x * m) >> 32) + x) >> l;
+#endif
+    }
+};
 
 // ---------------------------------------------------------------------------
 // status word: the first error wins
@@ -118,10 +143,28 @@ __device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c
 // quotient within one ulp of a/b, whose residual a - b q is then exact in a
 // fused multiply-add; with y the correctly rounded reciprocal, the second
 // correction RN(q + (a - b q) y) is the correctly rounded quotient.
-__device__ __forceinline__ float div_rn_by_correction(float a, float b, float y) {
+// The residual is exact only while it is a multiple of 2^-149: with
+// |b| >= 2^-90 that holds for every quotient of magnitude 2^-12 or more,
+// which covers every rounding tie of E2M1 and of the E4M3 scale; a smaller
+// quotient can be one ulp off but still lies below 2^-11, under the first tie
+// of either, so its code is unchanged.  Below 2^-90 the residual underflows
+// and quotients next to a tie round to the wrong side.  Above 2^125 the
+// reciprocal would be subnormal.  Callers therefore divide by correction only
+// for divisors in [kCorrectionMinDivisor, kCorrectionMaxDivisor].
+// (Host-callable too, with the host's IEEE multiply and fused multiply-add,
+// so that a host test can check the method on many quotients.)
+constexpr float kCorrectionMinDivisor = 0x1p-90f;
+constexpr float kCorrectionMaxDivisor = 0x1p125f;
+__host__ __device__ __forceinline__ float div_rn_by_correction(float a, float b, float y) {
+#ifdef __CUDA_ARCH__
     const float q0 = __fmul_rn(a, y);
     const float q1 = __fmaf_rn(__fmaf_rn(-q0, b, a), y, q0);
     return __fmaf_rn(__fmaf_rn(-q1, b, a), y, q1);
+#else
+    const float q0 = a * y;
+    const float q1 = fmaf(fmaf(-q0, b, a), y, q0);
+    return fmaf(fmaf(-q1, b, a), y, q1);
+#endif
 }
 // The same for two dividends at once (yy = (y, y), nb = (-b, -b)); the
 // quotients come back with the signs of their dividends, zeros included.
@@ -165,9 +208,9 @@ __device__ __forceinline__ void load16(const void* x, int64_t elem, float (&v)[1
 
 // Quantize one micro-block: returns the scale byte, writes 8 packed bytes.
 // The codes are E2M1(RN(v / den)) element by element.  A block with a NaN or
-// an infinity, a saturated scale (amax / (6 s_tensor) > 448), or a den that is
-// zero, subnormal or near the ends of the fp32 range takes the IEEE division
-// and the comparison encoder; every other block divides by correction from
+// an infinity, a saturated scale (amax / (6 s_tensor) > 448), or a den outside
+// [2^-90, 2^125] (where division by correction is not exact) takes the IEEE
+// division and the comparison encoder; every other block divides by correction from
 // one reciprocal and encodes two elements per hardware conversion -- the same
 // codes, bit for bit.
 __device__ __forceinline__ uint32_t quantize_block(const float (&v)[16], float s_tensor, uint2& packed) {
@@ -184,7 +227,7 @@ __device__ __forceinline__ uint32_t quantize_block(const float (&v)[16], float s
     const float den = __fmul_rn(e4m3_to_float(sb), s_tensor);
     uint32_t lo = 0, hi = 0;
     // r <= 448 bounds every |v / den| near 6, far from overflow
-    if (!nan && r <= 448.0f && den >= 0x1p-125f && den <= 0x1p125f) {
+    if (!nan && r <= 448.0f && den >= kCorrectionMinDivisor && den <= kCorrectionMaxDivisor) {
         const float y = __frcp_rn(den);
         uint32_t byte[8];
         // copysignf: a zero quotient keeps the sign of its dividend (the

@@ -90,23 +90,9 @@ cudaError_t launch_calib(const void* x, bool f32, int64_t n, float* d_s_tensor, 
 }
 
 // ---------------------------------------------------------------------------
-// Index arithmetic.  Division by a launch-invariant divisor (T. Granlund and
-// P. Montgomery, "Division by Invariant Integers using Multiplication", 1994):
-// for 1 <= d < 2^31 and 0 <= x < 2^31, x / d = (umulhi(x, m) + x) >> l with
-// l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1 (mod 2^32).  A
-// runtime 32-bit division is a software routine of a few dozen instructions;
-// this is two.
+// Index arithmetic: item indices are decoded with FastDiv (invariant
+// divisors, nvfp4kv_device.cuh), never with a runtime division.
 // ---------------------------------------------------------------------------
-struct FastDiv {
-    uint32_t d, m, l;
-    FastDiv() = default;
-    __host__ explicit FastDiv(uint32_t d_) : d(d_), m(0), l(0) {
-        while ((1ull << l) < d) ++l;
-        m = (uint32_t)((((1ull << 32) * ((1ull << l) - d)) / d + 1) & 0xFFFFFFFFull);
-    }
-    __device__ __forceinline__ uint32_t div(uint32_t x) const { return (__umulhi(x, m) + x) >> l; }
-};
-
 // launch-invariant shape of a quantize (nblk = elements per row / block size,
 // a power of two)
 struct QShape {
@@ -163,7 +149,9 @@ struct QTable {
     bool d6_fast;
 };
 
-__device__ __forceinline__ bool correction_range(float d) { return d >= 0x1p-125f && d <= 0x1p125f; }
+__device__ __forceinline__ bool correction_range(float d) {
+    return d >= kCorrectionMinDivisor && d <= kCorrectionMaxDivisor;
+}
 
 // all threads of the CTA; a barrier follows
 __device__ __forceinline__ void build_qtable(QTable& tb, float st) {

@@ -83,6 +83,8 @@ def test_traffic_dropped_when_source_changes(tmp_path, monkeypatch):
     digest = bench.source_digest(bench.ATTN_SOURCES)
     (tmp_path / "profiles" / "t.json").write_text(json.dumps(
         {"source_digest": digest, "dram_bytes_per_launch": 123}))
-    assert bench.profiled_traffic("t.json") == 123
+    assert bench.profiled_traffic("t.json") == (123, None)
     (tmp_path / bench.ATTN_SOURCES[0]).write_text("kernel v2")
-    assert bench.profiled_traffic("t.json") is None
+    traffic, why = bench.profiled_traffic("t.json")
+    assert traffic is None and "changed since the capture" in why
+    assert bench.profiled_traffic("missing.json")[0] is None

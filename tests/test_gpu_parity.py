@@ -159,6 +159,62 @@ def test_quantize_wide_range_f32_bit_exact(nv):
         np.testing.assert_array_equal(plane.scales.cpu().numpy(), ks)
 
 
+def _e2m1_tie_blocks(st, n_tok, H, D, seed):
+    """fp32 rows [1][n_tok][H][D] whose 16-element blocks take an E4M3 scale
+    value V under the tensor scale st (one element is RN(RN(6 st) V), so the
+    block maximum over 6 st rounds to V), every other element being RN(t den)
+    or one of its four nearest neighbours, den = RN(V st) the block divisor
+    and t a rounding tie of the E2M1 grid: quotients within a few ulps of a
+    tie, where a misrounded division changes the code."""
+    rng = np.random.default_rng(seed)
+    st = np.float32(st)
+    n_blk = n_tok * H * D // 16
+    V = ((1.0 + rng.integers(0, 8, n_blk) / 8.0) * np.exp2(rng.integers(-6, 9, n_blk))).astype(np.float32)
+    V = np.minimum(V, np.float32(448.0))
+    den = V * st
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    t = ties[rng.integers(0, ties.size, (n_blk, 16))]
+    a = (t * den[:, None]).astype(np.float32)
+    a = (a.view(np.int32) + rng.integers(-2, 3, (n_blk, 16)).astype(np.int32)).view(np.float32)
+    a[np.arange(n_blk), rng.integers(0, 16, n_blk)] = (np.float32(6.0) * st) * V
+    a = np.where(rng.random((n_blk, 16)) < 0.5, -a, a).astype(np.float32)
+    return torch.from_numpy(a.reshape(1, n_tok, H, D).copy())
+
+
+@pytest.mark.parametrize("st", [3.1e-33, 7.3e-31, 1.7e-28, 0.37])
+def test_quantize_near_ties_tiny_tensor_scales_bit_exact(nv, st):
+    """Blocks whose divisor den lies far below 1 (down to about 2^-114, where
+    the residual of a division by correction would underflow) or near 1, with
+    elements next to E2M1 rounding ties: codes and scales equal the oracle's,
+    through the quantize-append kernel and the append of the fused
+    append + attention kernel."""
+    n_tok, H, D = 64, 2, 128
+    x = _e2m1_tie_blocks(st, n_tok, H, D, seed=int(st * 1e3) % 1000 + 7)
+    st32 = np.float32(st)
+    s = torch.tensor([st32], device="cuda")
+    plane = nv.KVPlane.allocate(1, H, n_tok, D)
+    nv.nvfp4_kv_quantize_append(x.cuda(), torch.zeros(1, dtype=torch.int32, device="cuda"), s, plane)
+    kc, ks = oracle.new_planes(1, H, n_tok, D)
+    assert oracle.quantize_append(x.numpy(), np.zeros(1, np.int32), st32, kc, ks) == 0
+    np.testing.assert_array_equal(plane.codes.cpu().numpy(), kc)
+    np.testing.assert_array_equal(plane.scales.cpu().numpy(), ks)
+    # the same rows as n_tok sequences of one new token each
+    xb = x.view(n_tok, 1, H, D).contiguous()
+    q = torch.randn(n_tok, 4 * H, D, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    kp = nv.KVPlane.allocate(n_tok, H, 16, D)
+    vp = nv.KVPlane.allocate(n_tok, H, 16, D)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    start = torch.zeros(n_tok, dtype=torch.int32, device="cuda")
+    out = nv.nvfp4_decode_attention_append(q.cuda(), xb.cuda(), xb.cuda(), start, kp, vp, s, s, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0 and bool(torch.isfinite(out).all())
+    kc, ks = oracle.new_planes(n_tok, H, 16, D)
+    assert oracle.quantize_append(xb.numpy(), np.zeros(n_tok, np.int32), st32, kc, ks) == 0
+    for p in (kp, vp):
+        np.testing.assert_array_equal(p.codes[:, :, :1].cpu().numpy(), kc[:, :, :1])
+        np.testing.assert_array_equal(p.scales[:, :, :1].cpu().numpy(), ks[:, :, :1])
+
+
 @pytest.mark.parametrize("D", [64, 128])
 def test_dequant_random_planes_bit_exact(nv, D):
     B, H, S = 2, 3, 64
