@@ -417,8 +417,9 @@ nvfp4_status nvfp4_prefill_attention(const void* q, nvfp4_dtype q_dtype, int C, 
     if (d_s_tensor_k == nullptr || d_s_tensor_v == nullptr || d_start_pos == nullptr)
         return NVFP4_ERR_INVALID_ARG;
     if (!(std::isfinite(softmax_scale)) || softmax_scale < 0.0f) return NVFP4_ERR_INVALID_ARG;
-    // the tensor-core prefill takes bf16 queries (exact in its f16 operand);
-    // an fp32 query would need a second f16 term and its shared memory
+    // the tensor-core prefill takes bf16 queries (exact in its f16 operand
+    // after a power-of-two row scaling, down to 2^-31 of the row maximum); an
+    // fp32 query would need a second f16 term and its shared memory
     if (k->D != 128 || H_q / k->H_kv > 128 || q_dtype != NVFP4_IN_BF16) return NVFP4_ERR_UNSUPPORTED;
     if (k->B == 0 || C == 0) return NVFP4_OK;
     if (q == nullptr || out == nullptr || !aligned16(q) || !aligned16(out)) return NVFP4_ERR_INVALID_ARG;

@@ -271,8 +271,10 @@ nvfp4_status nvfp4_decode_attention(const void* q, nvfp4_dtype q_dtype, int H_q,
  * start_pos[b] + C - 1, attends causally: query i of sequence b sees the
  * cache tokens t <= start_pos[b] + i.  Runs on the tensor cores (tcgen05,
  * f16 MMAs with fp32 accumulation; the cache's FP8 values are exact in f16,
- * and so is a bf16 query after a power-of-two row scaling; the
- * probabilities enter as two f16 terms, about 22 significant bits).
+ * and so is a bf16 query after a power-of-two row scaling, for every element
+ * at least 2^-31 times the row's largest magnitude (smaller ones are rounded
+ * to f16's subnormal grid); the probabilities enter as two f16 terms, about
+ * 22 significant bits).
  *   q           device [B][C][H_q][128] bf16, 16-byte aligned (fp32 queries:
  *               NVFP4_ERR_UNSUPPORTED)
  *   C           chunk length (0: nothing to do)
