@@ -1,9 +1,13 @@
 """Host-side logic of bench.py on the CPU: the multi-rank reduction (gloo,
-world size 2), replica sizing against L2, clock-log parsing and the guard
-that drops profiled DRAM traffic once the kernel source changes."""
+world size 2), replica sizing against L2, clock-log parsing, the guard
+that drops profiled DRAM traffic once the kernel source changes, and the
+reference arm (the oracle on the host cores), which needs no GPU: its one
+JSON line at one rank and under torchrun at two."""
 import json
 import os
 import socket
+import subprocess
+import sys
 
 import pytest
 import torch
@@ -88,3 +92,41 @@ def test_traffic_dropped_when_source_changes(tmp_path, monkeypatch):
     traffic, why = bench.profiled_traffic("t.json")
     assert traffic is None and "changed since the capture" in why
     assert bench.profiled_traffic("missing.json")[0] is None
+
+
+REF_KEYS = {"impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+            "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"}
+
+
+def _check_reference_line(line, n):
+    d = json.loads(line)
+    assert REF_KEYS <= set(d), REF_KEYS - set(d)
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["n_gpus"] == n and d["steps"] == 1 and d["warmup"] == 3 and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["ms_per_step"] > 0 and d["vs_baseline"] is None
+    assert d["config"]["workload"].startswith(bench.DEFAULT_WORKLOAD)
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def _run(cmd):
+    r = subprocess.run(cmd, cwd=bench.ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    return lines
+
+
+def test_reference_arm_one_rank_prints_its_line():
+    lines = _run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3"])
+    assert len(lines) == 1
+    _check_reference_line(lines[0], 1)
+
+
+def test_reference_arm_under_torchrun_rank0_alone_prints():
+    lines = _run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                  "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py",
+                  "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"])
+    assert len(lines) == 1
+    _check_reference_line(lines[0], 2)
