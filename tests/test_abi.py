@@ -198,3 +198,22 @@ def test_header_is_plain_c_and_links(lib, tmp_path):
     assert int(out[0]) == 2 * 8 * 4096 * (64 + 8)
     assert int(out[1]) == 2 * 8 * 4096 * (64 + 4)
     assert len(out) > 2
+
+
+def test_missing_library_raises_and_cpu_tensors_are_refused(lib, monkeypatch):
+    # no CPU path: without the built library every call raises, and host
+    # tensors are refused before anything reaches the library
+    import torch
+
+    import bit_decode_attention_b200 as nv
+    monkeypatch.setattr(_native, "_lib", None)
+    monkeypatch.setattr(_native, "LIB_PATH", os.path.join(ROOT, "no", "such", "libnvfp4kv.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        _native.lib()
+    monkeypatch.undo()
+    x = torch.zeros(1, 1, 1, 128, dtype=torch.bfloat16)
+    plane = nv.KVPlane(torch.zeros(1, 1, 16, 64, dtype=torch.uint8), torch.zeros(1, 1, 16, 8, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="CUDA"):
+        nv.nvfp4_kv_quantize_append(x, torch.zeros(1, dtype=torch.int32), torch.ones(1), plane)
+    with pytest.raises(ValueError, match="CUDA"):
+        nv.nvfp4_calib_tensor_scale(x)
