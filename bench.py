@@ -98,8 +98,9 @@ def profiled_traffic(name):
     except Exception:
         return None, "no ncu capture of this workload under profiles/"
     if d.get("source_digest") != source_digest(ATTN_SOURCES):
-        return None, ("kernel sources changed since the capture in profiles/%s (digest %s); "
-                      "not re-captured" % (name, d.get("source_digest")))
+        return None, ("kernel sources changed since the capture in profiles/%s (digest %s, %s DRAM "
+                      "bytes per launch then); not re-captured"
+                      % (name, d.get("source_digest"), d.get("dram_bytes_per_launch")))
     return d.get("dram_bytes_per_launch"), None
 
 
