@@ -5,6 +5,8 @@ ml_dtypes float4_e2m1fn, torch scaled_dot_product_attention), closed forms,
 invariants and special cases.  CPU only.
 """
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import ml_dtypes
 import numpy as np
@@ -59,6 +61,28 @@ def test_e2m1_encode_matches_ml_dtypes():
     np.testing.assert_array_equal(mine, lib)
 
 
+def test_e2m1_encode_matches_ml_dtypes_on_every_nonnegative_float():
+    # exhaustive: every fp32 bit pattern from +0 to +inf (2.14e9 values)
+    # against ml_dtypes' cast, which rounds to nearest even and saturates at 6
+    # as the oracle does; chunks run over the host cores (both calls release
+    # the interpreter lock); negative values are in the sampled sweep above
+    # and the block sign-symmetry invariant
+    top = int(np.float32(np.inf).view(np.uint32)) + 1
+    chunk = 1 << 24
+
+    def compare(first):
+        bits = np.arange(first, min(first + chunk, top), dtype=np.uint32)
+        v = bits.view(np.float32)
+        mine = oracle.e2m1_encode(v)
+        lib = v.astype(ml_dtypes.float4_e2m1fn).view(np.uint8)
+        bad = np.flatnonzero(mine != lib)
+        return bad.size, [(hex(int(bits[i])), int(mine[i]), int(lib[i])) for i in bad[:5]]
+
+    with ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as pool:
+        results = list(pool.map(compare, range(0, top, chunk)))
+    assert sum(n for n, _ in results) == 0, [ex for n, ex in results if n][:3]
+
+
 def test_e2m1_ties_to_even_and_saturation():
     v = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.5, 1e9, -0.1, -0.0], np.float32)
     assert list(oracle.e2m1_encode(v)) == [0, 2, 2, 4, 4, 6, 6, 7, 7, 8, 8]
@@ -92,6 +116,28 @@ def test_e4m3_encode_matches_torch_below_saturation():
     mine = oracle.e4m3_encode(v)
     lib = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     np.testing.assert_array_equal(mine, lib)
+
+
+def test_e4m3_encode_matches_torch_on_every_float_below_464():
+    # exhaustive: every fp32 bit pattern in [0, 464) -- 1.14e9 values, every
+    # subnormal, tie and binade of the E4M3 range -- against torch's cast, in
+    # chunks over the host cores (both calls release the interpreter lock);
+    # from 464 up torch gives NaN where the oracle saturates (next test), and
+    # negative values are in the sampled sweep above
+    top = int(np.float32(464.0).view(np.uint32))
+    chunk = 1 << 24
+
+    def compare(first):
+        bits = np.arange(first, min(first + chunk, top), dtype=np.uint32)
+        v = bits.view(np.float32)
+        mine = oracle.e4m3_encode(v)
+        lib = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        bad = np.flatnonzero(mine != lib)
+        return bad.size, [(hex(int(bits[i])), int(mine[i]), int(lib[i])) for i in bad[:5]]
+
+    with ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as pool:
+        results = list(pool.map(compare, range(0, top, chunk)))
+    assert sum(n for n, _ in results) == 0, [ex for n, ex in results if n][:3]
 
 
 def test_e4m3_satfinite():
