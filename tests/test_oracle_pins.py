@@ -386,6 +386,23 @@ def test_attention_special_cases():
     np.testing.assert_allclose(out[0, 0, :2], [2 * w0, 1 - w0], rtol=1e-14)
 
 
+def test_attention_one_dominant_score_returns_its_row():
+    # one token's score exceeds every other by ~1.1e4: its softmax weight is
+    # 1 and the others' exp(-1.1e4) are 0 in fp64, so the output is that V row
+    rng = np.random.default_rng(23)
+    B, H_q, H_kv, S, D = 1, 1, 1, 50, 16
+    _, v8 = _rand_fp8_planes(rng, B, H_kv, S, D)
+    v8 = _sanitize(v8)
+    V = _fp8_values(v8).numpy()
+    for j in (0, 17, S - 1):
+        k8 = np.zeros((B, H_kv, S, D), np.uint8)
+        k8[0, 0, j, 0] = 0x7E                  # k_j = 448 e0, every other key 0
+        q = np.zeros((B, H_q, D), np.float32)
+        q[0, 0, 0] = 100.0
+        out = oracle.decode_attention_fp8(q, k8, v8, np.array([S], np.int32))
+        np.testing.assert_array_equal(out[0, 0], V[0, 0, j])
+
+
 def test_attention_token_permutation_invariance():
     rng = np.random.default_rng(19)
     B, H_q, H_kv, S, D = 1, 4, 2, 30, 16
