@@ -487,15 +487,15 @@ def roofline_block(wl, att_ms, att_n, peak, peak_kind, traffic_name=None):
     g = wl.w.Hq // wl.w.Hkv
     traffic, why = profiled_traffic(traffic_name) if traffic_name else (None, "no capture named")
     block = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak,
-            "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-            else "fallback",
-            "traffic": traffic,
-            "kernel": "decode_attention_tc_kernel<%d> + merge_split_units_kernel (tcgen05, head_dim "
-                      "128, bf16 queries, GQA group %d)" % (1 if g <= 8 else 2, g),
-            "algorithmic_bytes_per_launch": wl.attention_bytes(),
-            "launch_ms": att_ms, "launches_sampled": att_n,
-            "frac_of_nominal_8tbs": achieved / 8000.0}
+             "frac": achieved / peak,
+             "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+             else "fallback",
+             "traffic": traffic,
+             "kernel": "decode_attention_tc_kernel<%d> + merge_split_units_kernel (tcgen05, head_dim "
+                       "128, bf16 queries, GQA group %d)" % (1 if g <= 8 else 2, g),
+             "algorithmic_bytes_per_launch": wl.attention_bytes(),
+             "launch_ms": att_ms, "launches_sampled": att_n,
+             "frac_of_nominal_8tbs": achieved / 8000.0}
     if why:
         block["traffic_note"] = why
     return block
