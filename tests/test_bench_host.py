@@ -118,12 +118,14 @@ def _run(cmd):
     return lines
 
 
+@pytest.mark.slow
 def test_reference_arm_one_rank_prints_its_line():
     lines = _run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3"])
     assert len(lines) == 1
     _check_reference_line(lines[0], 1)
 
 
+@pytest.mark.slow
 def test_reference_arm_under_torchrun_rank0_alone_prints():
     lines = _run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
                   "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py",

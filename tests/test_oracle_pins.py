@@ -61,6 +61,7 @@ def test_e2m1_encode_matches_ml_dtypes():
     np.testing.assert_array_equal(mine, lib)
 
 
+@pytest.mark.slow
 def test_e2m1_encode_matches_ml_dtypes_on_every_nonnegative_float():
     # exhaustive: every fp32 bit pattern from +0 to +inf (2.14e9 values)
     # against ml_dtypes' cast, which rounds to nearest even and saturates at 6
@@ -118,6 +119,7 @@ def test_e4m3_encode_matches_torch_below_saturation():
     np.testing.assert_array_equal(mine, lib)
 
 
+@pytest.mark.slow
 def test_e4m3_encode_matches_torch_on_every_float_below_464():
     # exhaustive: every fp32 bit pattern in [0, 464) -- 1.14e9 values, every
     # subnormal, tie and binade of the E4M3 range -- against torch's cast, in
